@@ -1,0 +1,223 @@
+// Shared internals of the sm_100a library behind include/sla.h: error
+// reporting, the CSR handle, and device helpers (deterministic reductions and
+// a bounded device-wide barrier for persistent cooperative kernels).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/sla.h"
+
+namespace sla {
+
+// ---------------------------------------------------------------- errors ----
+void set_error(const char *fmt, ...);
+void clear_error();
+
+#define SLA_CHECK_CUDA(call)                                                   \
+    do {                                                                       \
+        cudaError_t e_ = (call);                                               \
+        if (e_ != cudaSuccess) {                                               \
+            ::sla::set_error("%s failed: %s (%s:%d)", #call,                   \
+                             cudaGetErrorString(e_), __FILE__, __LINE__);      \
+            return SLA_ERR_CUDA;                                               \
+        }                                                                      \
+    } while (0)
+
+#define SLA_CHECK_LAUNCH()                                                     \
+    do {                                                                       \
+        cudaError_t e_ = cudaGetLastError();                                   \
+        if (e_ != cudaSuccess) {                                               \
+            ::sla::set_error("kernel launch failed: %s (%s:%d)",               \
+                             cudaGetErrorString(e_), __FILE__, __LINE__);      \
+            return SLA_ERR_CUDA;                                               \
+        }                                                                      \
+    } while (0)
+
+#define SLA_REQUIRE(cond, ...)                                                 \
+    do {                                                                       \
+        if (!(cond)) {                                                         \
+            ::sla::set_error(__VA_ARGS__);                                     \
+            return SLA_ERR_INVALID;                                            \
+        }                                                                      \
+    } while (0)
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+// Sequential carving of a caller workspace into 256-byte aligned pieces.
+struct Carver {
+    char *base;
+    size_t off = 0;
+    explicit Carver(void *p) : base(static_cast<char *>(p)) {}
+    template <typename U>
+    U *take(size_t count) {
+        U *p = reinterpret_cast<U *>(base ? base + off : nullptr);
+        off = align_up(off + count * sizeof(U));
+        return p;
+    }
+};
+
+// Rows handled by one thread block in row-parallel kernels.
+constexpr int kRowBlock = 256;
+// Threads of the persistent-grid and block-per-system CG kernels.
+constexpr int kCgThreads = 512;
+
+// ---------------------------------------------------------------- handle ----
+struct Csr {
+    int32_t n_rows = 0, n_cols = 0;
+    int64_t nnz = 0;
+    int32_t batch = 1;
+    sla_dtype dtype = SLA_F64;
+    uint32_t flags = 0;
+    int device = 0;
+    int num_sms = 0;
+    const int32_t *rowptr = nullptr;   // borrowed
+    const int32_t *colind = nullptr;   // borrowed
+    int32_t *diagpos = nullptr;        // owned [n_rows]: position of A_ii, -1 if absent
+    // A^T's pattern (owned; built on request)
+    int32_t *rowptrT = nullptr, *colindT = nullptr, *permT = nullptr, *diagposT = nullptr;
+    bool has_transpose = false;
+    // statistics
+    int32_t row_min = 0, row_max = 0;
+    double row_mean = 0.0;
+    int32_t lanes = 1;
+    // persistent-grid CG layout
+    int32_t grid_blocks = 0;           // cooperative grid size for this dtype
+    int32_t tile_rows = 0;             // rows of one tile (tiles never straddle systems)
+    int32_t ntiles = 0;                // tiles per system
+    bool block_fits = false;           // one system fits the block-per-system solver
+    size_t block_smem = 0;             // its dynamic shared memory per block
+};
+
+inline size_t dtype_size(sla_dtype dt) { return dt == SLA_F64 ? 8 : 4; }
+
+// Picks the threads-per-row of row-parallel kernels from the mean row length.
+int lanes_for_mean(double mean_row);
+
+// Builds A^T's pattern into the handle (allocates once).
+sla_status ensure_transpose(Csr *h, cudaStream_t s);
+
+// Stable radix-sort based transpose of a pattern; used by the public call and
+// the handle.  `ws` must hold transpose_ws_bytes().
+size_t transpose_ws_bytes(int32_t n_rows, int32_t n_cols, int64_t nnz);
+sla_status transpose_pattern(int32_t n_rows, int32_t n_cols, int64_t nnz,
+                             const int32_t *rowptr, const int32_t *colind,
+                             int32_t *rowptrT, int32_t *colindT, int32_t *perm,
+                             void *ws, cudaStream_t s);
+
+// valsT[b][s] = vals[b][permT[s]] for every system (needs the handle's A^T).
+sla_status transpose_values(const Csr *h, const void *vals, void *valsT, cudaStream_t s);
+
+// Diagonal positions of a square pattern (kernel; enqueue only).
+sla_status diag_positions(int32_t n, const int32_t *rowptr, const int32_t *colind,
+                          int32_t *diagpos, cudaStream_t s);
+
+// ------------------------------------------------------- device helpers ----
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Deterministic block sum of one double per thread; every thread of the block
+// must call it.  The result is returned to all threads.  `red` holds >= 33
+// doubles of shared memory.
+template <int NT>
+__device__ __forceinline__ double block_sum(double v, double *red) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_sum(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        double s = lane < NW ? red[lane] : 0.0;
+        s = warp_sum(s);
+        if (lane == 0) red[32] = s;
+    }
+    __syncthreads();
+    const double r = red[32];
+    __syncthreads();
+    return r;
+}
+
+// Two sums in one pass (same order as two block_sum calls).
+template <int NT>
+__device__ __forceinline__ void block_sum2(double &a, double &b, double *red) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    a = warp_sum(a);
+    b = warp_sum(b);
+    if (lane == 0) { red[warp] = a; red[32 + warp] = b; }
+    __syncthreads();
+    if (warp == 0) {
+        double s = lane < NW ? red[lane] : 0.0;
+        double t = lane < NW ? red[32 + lane] : 0.0;
+        s = warp_sum(s);
+        t = warp_sum(t);
+        if (lane == 0) { red[64] = s; red[65] = t; }
+    }
+    __syncthreads();
+    a = red[64];
+    b = red[65];
+    __syncthreads();
+}
+
+// Device-wide barrier for a cooperative (co-resident) grid.  sync[0] counts
+// arrivals, sync[1] is the generation, sync[2] the error flag.  Each wait is
+// bounded by timeout_ns of %globaltimer; a block that gives up sets the error
+// flag, and blocks that see the flag give up too.  Returns false when the
+// caller must leave the kernel.  Every thread of the block must call it.
+__device__ __forceinline__ bool grid_barrier(unsigned *sync, unsigned nblocks,
+                                             long long timeout_ns, int *flag_smem) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned *count = sync, *gen = sync + 1, *err = sync + 2;
+        const unsigned g = ld_acquire_u32(gen);
+        int ok = 1;
+        __threadfence();
+        const unsigned prev = atomicAdd(count, 1u);
+        if (prev == nblocks - 1) {
+            atomicExch(count, 0u);
+            __threadfence();
+            atomicAdd(gen, 1u);
+        } else {
+            const unsigned long long t0 = global_timer_ns();
+            unsigned spins = 0;
+            while (ld_acquire_u32(gen) == g) {
+                if ((++spins & 31u) == 0) {
+                    if (ld_acquire_u32(err) != 0) { ok = 0; break; }
+                    if ((long long)(global_timer_ns() - t0) > timeout_ns) {
+                        atomicExch(err, 1u);
+                        ok = 0;
+                        break;
+                    }
+                }
+            }
+        }
+        if (ok && ld_acquire_u32(err) != 0) ok = 0;
+        __threadfence();
+        *flag_smem = ok;
+    }
+    __syncthreads();
+    return *flag_smem != 0;
+}
+
+}  // namespace sla

@@ -1,0 +1,73 @@
+// Row-parallel building blocks: one row of a CSR matrix times a vector, with
+// LANES threads of a warp cooperating on the row (LANES in 1..32, a power of
+// two).  Matrix arrays are read through the read-only path; the vector is read
+// with plain loads because the persistent solver rewrites it between phases.
+#pragma once
+
+#include "sla_common.cuh"
+
+namespace sla {
+
+template <int LANES>
+__device__ __forceinline__ unsigned subwarp_mask() {
+    if constexpr (LANES == 32) {
+        return 0xffffffffu;
+    } else {
+        const unsigned base = (threadIdx.x & 31) & ~(LANES - 1);
+        return ((1u << LANES) - 1u) << base;
+    }
+}
+
+// sum_{t in row i} vals[t] * v[colind[t]]; lane in [0, LANES).  With LANES > 1
+// the partial sums are combined by a fixed xor tree, so the result is
+// deterministic and identical on every lane of the sub-warp.
+template <typename T, int LANES>
+__device__ __forceinline__ T row_dot(const int32_t *__restrict__ rowptr,
+                                     const int32_t *__restrict__ colind,
+                                     const T *__restrict__ vals, const T *v, int i,
+                                     int lane) {
+    const int t0 = __ldg(rowptr + i), t1 = __ldg(rowptr + i + 1);
+    T s = T(0);
+    for (int t = t0 + lane; t < t1; t += LANES) s += __ldg(vals + t) * v[__ldg(colind + t)];
+    if constexpr (LANES > 1) {
+        const unsigned m = subwarp_mask<LANES>();
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) s += __shfl_xor_sync(m, s, o, LANES);
+    }
+    return s;
+}
+
+// Same with the values reached through a permutation (A^T's entry s is A's
+// entry perm[s]); used by transposed SpMV on non-symmetric handles.
+template <typename T, int LANES>
+__device__ __forceinline__ T row_dot_perm(const int32_t *__restrict__ rowptr,
+                                          const int32_t *__restrict__ colind,
+                                          const int32_t *__restrict__ perm,
+                                          const T *__restrict__ vals, const T *v, int i,
+                                          int lane) {
+    const int t0 = __ldg(rowptr + i), t1 = __ldg(rowptr + i + 1);
+    T s = T(0);
+    for (int t = t0 + lane; t < t1; t += LANES)
+        s += __ldg(vals + __ldg(perm + t)) * v[__ldg(colind + t)];
+    if constexpr (LANES > 1) {
+        const unsigned m = subwarp_mask<LANES>();
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) s += __shfl_xor_sync(m, s, o, LANES);
+    }
+    return s;
+}
+
+// Dispatch a functor templated on LANES.
+template <typename F>
+sla_status with_lanes(int lanes, F &&f) {
+    switch (lanes) {
+        case 1: return f(std::integral_constant<int, 1>{});
+        case 2: return f(std::integral_constant<int, 2>{});
+        case 4: return f(std::integral_constant<int, 4>{});
+        case 8: return f(std::integral_constant<int, 8>{});
+        case 16: return f(std::integral_constant<int, 16>{});
+        default: return f(std::integral_constant<int, 32>{});
+    }
+}
+
+}  // namespace sla

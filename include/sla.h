@@ -1,0 +1,267 @@
+/*
+ * sla.h -- C ABI of the B200 (sm_100a) library for differentiable sparse SPD
+ * solves on CSR matrices: Jacobi-preconditioned conjugate gradient, its
+ * implicit-function-theorem adjoint, and the sparse value gradient.
+ *
+ * The operations follow "torch-sla: Differentiable Sparse Linear Algebra with
+ * Adjoint Solvers and Sparse Tensor Parallelism for PyTorch" (gist.science
+ * summary page, technical summary):
+ *   - "Methodology" 1 (unified backend abstraction): the autograd-aware
+ *     `.solve` and `.matvec` calls, an iterative GPU solver, and the
+ *     `SparseTensor` type that holds one matrix or a batch sharing one pattern;
+ *   - "Methodology" 2 (adjoint differentiation framework, linear systems): the
+ *     backward pass solves one adjoint system A^T lambda = dL/dx, and the
+ *     gradient with respect to the matrix is -lambda_i * x_j on the sparsity
+ *     pattern only (dL/db = lambda follows from the same implicit-function
+ *     argument);
+ *   - "Significance" (limitations): the PyTorch-native iterative backend uses
+ *     a Jacobi preconditioner.
+ *
+ * Conventions shared by every call
+ *   - Indices are int32: rowptr[n_rows + 1], colind[nnz], so nnz < 2^31.
+ *     Column indices within a row are strictly increasing (validated by
+ *     SLA_FLAG_VALIDATE or sla_csr_check).
+ *   - Pointers named "device" must point to GPU global memory of the current
+ *     device; the caller allocates and frees them.  The library never keeps a
+ *     caller pointer beyond the call except rowptr/colind, which a handle
+ *     borrows: they must stay valid and unchanged until sla_csr_destroy.
+ *   - Batched arrays are batch-major and contiguous: values [B][nnz],
+ *     vectors [B][n].  All B systems share the handle's pattern.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns; results are valid once the stream
+ *     reaches that point.  No call synchronises the host except
+ *     sla_csr_create (pattern analysis) and the one-time lazy build of A^T's
+ *     pattern (first transposed use of a non-symmetric handle).
+ *   - Calls return an sla_status synchronously for argument errors and CUDA
+ *     launch errors; sla_last_error_string() (per host thread) explains the
+ *     last non-OK status.  Solve outcomes are per system and written to device
+ *     memory (sla_cg_info) because they are only known on the GPU.
+ *   - Workspace is caller-provided device memory of at least
+ *     sla_workspace_bytes() bytes, 256-byte aligned.  Solves and SpMVs never
+ *     allocate device memory.  Concurrent calls need distinct workspaces.
+ *   - Every device-side wait is bounded (sla_cg_opts.wait_timeout_ns); a wait
+ *     that runs out makes the kernel return and the affected systems report
+ *     SLA_TIMED_OUT.  No kernel traps.
+ */
+#ifndef SLA_H
+#define SLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sla_csr_s *sla_csr_t;
+
+typedef enum { SLA_F64 = 0, SLA_F32 = 1 } sla_dtype;
+
+/* Call-level status. */
+typedef enum {
+    SLA_OK = 0,
+    SLA_ERR_INVALID = 1,      /* bad argument or invalid pattern */
+    SLA_ERR_CUDA = 2,         /* a CUDA runtime call or launch failed */
+    SLA_ERR_OOM = 3,          /* sla_csr_create could not allocate its metadata */
+    SLA_ERR_TIMEOUT = 4,      /* reserved for host-side waits */
+    SLA_ERR_UNSUPPORTED = 5   /* valid request this build cannot serve */
+} sla_status;
+
+/* Per-system solve outcome (device int32 in sla_cg_info.status). */
+enum {
+    SLA_CONVERGED = 0,        /* ||r_k|| <= max(rtol ||b||, atol), or r_k == 0 */
+    SLA_NOT_CONVERGED = 1,    /* max_iter reached in tolerance mode */
+    SLA_BREAKDOWN = 2,        /* p.Ap <= 0, or a diagonal entry <= 0 under Jacobi */
+    SLA_NONFINITE = 3,        /* NaN/Inf in b, p.Ap or ||r||^2 */
+    SLA_FIXED_DONE = 4,       /* exactly fixed_iters iterations ran */
+    SLA_TIMED_OUT = 5         /* a device-side wait ran out; x is not valid */
+};
+
+/* sla_csr_create flags. */
+enum {
+    SLA_FLAG_VALIDATE = 1u,        /* check the pattern (sync); invalid -> SLA_ERR_INVALID */
+    SLA_FLAG_SYMMETRIC = 2u,       /* caller asserts A^T == A for every value set */
+    SLA_FLAG_BUILD_TRANSPOSE = 4u  /* build A^T's pattern now (needed for transposed ops
+                                      on a non-symmetric handle; built lazily otherwise) */
+};
+
+/* Solver strategies (sla_cg_opts.strategy).  AUTO picks by size: one thread
+ * block per system when a system's vectors fit in shared memory, else one
+ * persistent cooperative grid with device-wide barriers.  The others force a
+ * choice (benchmarks and tests). */
+enum { SLA_STRATEGY_AUTO = 0, SLA_STRATEGY_GRID = 1, SLA_STRATEGY_BLOCK = 2 };
+
+typedef struct {
+    double rtol;              /* relative residual target (tolerance mode) */
+    double atol;              /* absolute residual floor; stop at max(rtol*||b||, atol) */
+    int32_t max_iter;         /* cap in tolerance mode; <= 0 means min(10 n, 100000) */
+    int32_t fixed_iters;      /* > 0: run exactly this many iterations, no tolerance test */
+    int32_t precond;          /* 1: Jacobi M = diag(A); 0: none */
+    int32_t x0_given;         /* 1: x holds the initial guess on entry; 0: start from 0 */
+    int64_t wait_timeout_ns;  /* bound on each device-side wait; <= 0 means 5 s */
+    int32_t strategy;         /* SLA_STRATEGY_* */
+    int32_t reserved;         /* must be 0 */
+} sla_cg_opts;
+
+/* Per-system outputs, device pointers to [B] arrays; any may be NULL. */
+typedef struct {
+    int32_t *iters;           /* completed iterations (alpha-updates) */
+    double *relres;           /* recursive ||r_k|| / ||b|| at exit */
+    int32_t *status;          /* SLA_CONVERGED ... SLA_TIMED_OUT */
+} sla_cg_info;
+
+/* Pattern statistics a handle computed at creation (host copy). */
+typedef struct {
+    int32_t n_rows, n_cols;
+    int64_t nnz;
+    int32_t batch;
+    int32_t dtype;            /* sla_dtype */
+    int32_t row_min, row_max; /* entries per row */
+    double row_mean;
+    int32_t lanes;            /* threads cooperating on one row in SpMV-like kernels */
+    int32_t grid_blocks;      /* persistent-grid size on this device */
+    int32_t block_fits;       /* 1 if one system fits the block-per-system solver */
+    int32_t has_transpose;    /* 1 once A^T's pattern is built */
+} sla_csr_props;
+
+/* Operations for sla_workspace_bytes. */
+enum { SLA_OP_SPMV = 0, SLA_OP_CG = 1, SLA_OP_ADJOINT = 2, SLA_OP_GRAD = 3 };
+
+/*
+ * Create a handle for a CSR pattern shared by `batch` value sets of `dtype`
+ * ("Methodology" 1: SparseTensor with one shared pattern).
+ * rowptr/colind: device, borrowed until destroy.  The handle allocates and owns
+ * derived metadata only (diagonal positions; A^T's pattern when requested).
+ * Synchronises `stream` once to read the pattern statistics (and the check
+ * result with SLA_FLAG_VALIDATE).  Errors: SLA_ERR_INVALID (sizes, NULL,
+ * invalid pattern with VALIDATE; the message names the first bad index),
+ * SLA_ERR_OOM, SLA_ERR_CUDA.  *out is NULL on error.
+ */
+sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz,
+                          const int32_t *rowptr, const int32_t *colind,
+                          int32_t batch, sla_dtype dtype, uint32_t flags,
+                          void *stream, sla_csr_t *out);
+
+/* Release a handle and its metadata (waits for nothing; the caller must not
+ * destroy a handle that queued work still uses).  NULL is a no-op. */
+sla_status sla_csr_destroy(sla_csr_t h);
+
+/* Host copy of the handle's statistics. */
+sla_status sla_csr_get_props(sla_csr_t h, sla_csr_props *props);
+
+/* Device pointers to A^T's pattern and the value permutation (A^T's entry s is
+ * A's entry perm[s]); builds them on `stream` if not built yet.  Valid until
+ * destroy.  For square symmetric handles the pattern equals A's. */
+sla_status sla_csr_transpose_pattern(sla_csr_t h, const int32_t **rowptrT,
+                                     const int32_t **colindT, const int32_t **perm,
+                                     void *stream);
+
+/* Workspace bytes that `op` needs on this handle (0 if none). */
+size_t sla_workspace_bytes(sla_csr_t h, int32_t op);
+
+/*
+ * Batched SpMV ("Methodology" 1, `.matvec`):
+ *   y_b = alpha * op(A_b) x_b + beta * y_b,  op = A (transpose == 0) or A^T.
+ * vals: device [B][nnz]; x: device [B][n_cols] (A) or [B][n_rows] (A^T);
+ * y: device [B][n_rows] or [B][n_cols].  beta == 0 never reads y.  x and y must
+ * not overlap.  A^T on a non-symmetric handle uses A^T's pattern (built here on
+ * first use, which allocates handle metadata once).
+ */
+sla_status sla_spmv(sla_csr_t h, const void *vals, const void *x, void *y,
+                    int32_t transpose, double alpha, double beta, void *stream);
+
+/*
+ * Batched Jacobi-preconditioned CG solve of A_b x_b = b_b for every system b
+ * (the iterative `.solve` of "Methodology" 1 with the Jacobi preconditioner
+ * of "Significance").  Textbook Hestenes-Stiefel PCG; stopping on the
+ * recursively updated residual; fixed mode runs exactly fixed_iters steps.
+ * For dtype F32, vectors and row sums are fp32 and every dot product is
+ * accumulated in fp64.  Each system stops on its own; the whole iteration
+ * runs on the GPU with no host synchronisation.
+ * vals [B][nnz], b [B][n], x [B][n] (in: initial guess if x0_given; out:
+ * solution), all device.  ws: device, >= sla_workspace_bytes(h, SLA_OP_CG).
+ * Requires n_rows == n_cols.
+ */
+sla_status sla_cg_solve(sla_csr_t h, const void *vals, const void *b, void *x,
+                        const sla_cg_opts *opts, sla_cg_info info,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Adjoint solve A_b^T lambda_b = g_b ("Methodology" 2, linear systems: the
+ * backward pass solves one adjoint system with right-hand side dL/dx).  With
+ * SLA_FLAG_SYMMETRIC the forward pattern and values are used as they are;
+ * otherwise A^T's values are gathered into the workspace first.
+ * Same arguments and outcomes as sla_cg_solve (lambda plays x; dL/db = lambda).
+ * ws >= sla_workspace_bytes(h, SLA_OP_ADJOINT).
+ */
+sla_status sla_cg_adjoint(sla_csr_t h, const void *vals, const void *g, void *lambda,
+                          const sla_cg_opts *opts, sla_cg_info info,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Sparse value gradient ("Methodology" 2: dL/dA_ij = -lambda_i x_j on the
+ * sparsity pattern only):  grad_b[t] = -lambda_b[i] * x_b[colind[t]] for entry
+ * t of row i, or grad_b[t] += that value when accumulate != 0.
+ * lambda [B][n_rows], x [B][n_cols], grad [B][nnz]; device.
+ */
+sla_status sla_grad_values(sla_csr_t h, const void *lambda, const void *x, void *grad,
+                           int32_t accumulate, void *stream);
+
+/*
+ * Transpose of a batched CSR matrix by a stable sort on the column index:
+ * row c of A^T lists the entries of column c in increasing row order; values
+ * are moved, never combined; perm[s] is the A-position of A^T's entry s.
+ * Inputs device: rowptr[n_rows+1], colind[nnz], vals [B][nnz] (may be NULL to
+ * skip values).  Outputs device: rowptrT[n_cols+1], colindT[nnz], valsT
+ * [B][nnz] (ignored if vals is NULL), perm[nnz] (may be NULL only when vals
+ * is NULL).  ws >= sla_transpose_workspace_bytes().  Bit-exact by
+ * construction.  The pattern must be valid (see sla_csr_check).
+ */
+size_t sla_transpose_workspace_bytes(int32_t n_rows, int32_t n_cols, int64_t nnz);
+sla_status sla_csr_transpose(int32_t n_rows, int32_t n_cols, int64_t nnz,
+                             const int32_t *rowptr, const int32_t *colind,
+                             int32_t batch, sla_dtype dtype, const void *vals,
+                             int32_t *rowptrT, int32_t *colindT, void *valsT,
+                             int32_t *perm, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * CSR from coordinate entries: entries ordered by (row, col) with a stable
+ * sort; runs of equal (row, col) are summed left to right in input order.
+ * Inputs device: row[nnz_in], col[nnz_in], val [B][nnz_in] (may be NULL).
+ * Outputs device: rowptr[n_rows+1], colind[capacity nnz_in], val_out
+ * [B][nnz_in] (row stride nnz_in; first *nnz_out entries of each row used),
+ * slot[nnz_in] (output position of each input entry; may be NULL),
+ * nnz_out (device int64[1]).  ws >= sla_coo_workspace_bytes().  Entries out of
+ * range make the call write -1 to *nnz_out and leave the outputs undefined.
+ */
+size_t sla_coo_workspace_bytes(int32_t n_rows, int32_t n_cols, int64_t nnz_in);
+sla_status sla_csr_from_coo(int32_t n_rows, int32_t n_cols, int64_t nnz_in,
+                            const int32_t *row, const int32_t *col,
+                            int32_t batch, sla_dtype dtype, const void *val,
+                            int32_t *rowptr, int32_t *colind, void *val_out,
+                            int32_t *slot, int64_t *nnz_out,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Pattern check on the GPU.  result: device int64[2] receives {code, where}:
+ * 0 valid; 1 rowptr[0] != 0; 2 rowptr decreases at row `where`; 3 rowptr[n_rows]
+ * != nnz; 4 column out of range at entry `where`; 5 columns not strictly
+ * increasing at entry `where`; 6 (need_diag) row `where` has no diagonal.
+ * When several problems exist, the lowest code wins and, within it, the lowest
+ * index.  Enqueue-only.
+ */
+sla_status sla_csr_check(int32_t n_rows, int32_t n_cols, int64_t nnz,
+                         const int32_t *rowptr, const int32_t *colind,
+                         int32_t need_diag, int64_t *result, void *stream);
+
+/* Message for the last non-OK status on this host thread ("" if none). */
+const char *sla_last_error_string(void);
+
+/* Library version string. */
+const char *sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H */

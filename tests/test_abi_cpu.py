@@ -1,0 +1,76 @@
+"""The C-ABI library loads and exports every declared entry point; host-side
+argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from differentiable_sparse_linear_csr_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "sla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sla_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary_calls():
+    names = _declared_functions()
+    for required in ("sla_csr_create", "sla_spmv", "sla_cg_solve", "sla_cg_adjoint",
+                     "sla_grad_values", "sla_csr_transpose", "sla_csr_from_coo"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = L.lib()
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(_declared_functions()) <= set(L._SIGNATURES), "binding lacks a declared call"
+
+
+def test_version_and_error_string():
+    assert "sm_100a" in L.sla_version()
+    assert isinstance(L.sla_last_error_string(), str)
+
+
+def test_host_side_argument_errors_need_no_gpu():
+    lib = L.lib()
+    h = ctypes.c_void_p()
+    st = lib.sla_csr_create(4, 4, 8, None, None, 1, 0, 0, None, ctypes.byref(h))
+    assert st == L.SLA_ERR_INVALID and h.value is None
+    assert "rowptr" in L.sla_last_error_string()
+    st = lib.sla_csr_create(-1, 4, 0, ctypes.c_void_p(256), None, 1, 0, 0, None, ctypes.byref(h))
+    assert st == L.SLA_ERR_INVALID
+    st = lib.sla_csr_create(4, 4, 0, ctypes.c_void_p(256), None, 0, 0, 0, None, ctypes.byref(h))
+    assert st == L.SLA_ERR_INVALID and "batch" in L.sla_last_error_string()
+    st = lib.sla_csr_create(4, 4, 0, ctypes.c_void_p(256), None, 1, 7, 0, None, ctypes.byref(h))
+    assert st == L.SLA_ERR_INVALID and "dtype" in L.sla_last_error_string()
+    st = lib.sla_csr_create(4, 5, 0, ctypes.c_void_p(256), None, 1, 0, L.SLA_FLAG_SYMMETRIC, None,
+                            ctypes.byref(h))
+    assert st == L.SLA_ERR_INVALID and "square" in L.sla_last_error_string()
+    assert lib.sla_spmv(None, None, None, None, 0, 1.0, 0.0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_grad_values(None, None, None, None, 0, None) == L.SLA_ERR_INVALID
+    opts = L.make_opts()
+    info = L.make_info()
+    assert lib.sla_cg_solve(None, None, None, None, ctypes.byref(opts), info, None, 0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_cg_adjoint(None, None, None, None, ctypes.byref(opts), info, None, 0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_workspace_bytes(None, L.SLA_OP_CG) == 0
+    assert lib.sla_csr_destroy(None) == L.SLA_OK
+
+
+def test_workspace_sizes_grow_with_size():
+    a = L.sla_transpose_workspace_bytes(100, 100, 1000)
+    b = L.sla_transpose_workspace_bytes(100_000, 100_000, 1_000_000)
+    assert 0 < a < b
+    assert L.sla_coo_workspace_bytes(10, 10, 100) > 0
+    assert L.sla_transpose_workspace_bytes(-1, 1, 1) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "_LIB_PATH", str(tmp_path / "libsla.so"))
+    with pytest.raises(ImportError, match="missing"):
+        L.lib()
