@@ -202,7 +202,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned *sync, unsigned nblocks,
             const unsigned long long t0 = global_timer_ns();
             unsigned spins = 0;
             while (ld_acquire_u32(gen) == g) {
-                if ((++spins & 31u) == 0) {
+                if ((spins++ & 7u) == 0) {   // first poll, then every 8th
                     if (ld_acquire_u32(err) != 0) { ok = 0; break; }
                     if ((long long)(global_timer_ns() - t0) > timeout_ns) {
                         atomicExch(err, 1u);

@@ -385,7 +385,7 @@ def test_adjoint_memory_does_not_grow_with_iterations():
     b = T(W.normal(1, 0, 200 * 200))
     vals = T(v)
     peaks = []
-    for k in (10, 1000):
+    for k in (10, 10, 1000):   # the first pass warms up library-independent allocations
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats()
         base = torch.cuda.memory_allocated()
@@ -395,7 +395,7 @@ def test_adjoint_memory_does_not_grow_with_iterations():
         torch.cuda.synchronize()
         peaks.append(torch.cuda.max_memory_allocated() - base)
         del x, vv
-    assert peaks[0] == peaks[1]
+    assert peaks[1] == peaks[2]
 
 
 # ------------------------------------------------------------ edge cases ----
