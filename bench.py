@@ -1,0 +1,366 @@
+"""Benchmark of the differentiable sparse SPD solve on B200.
+
+One step = the whole hot path on the 2-D 5-point Poisson system on a 1024x1024
+grid (n = 1,048,576, nnz = 5,238,784): a fixed 1000-iteration Jacobi-PCG
+forward solve, the 1000-iteration adjoint solve A^T lambda = x - x*, and the
+sparse value gradient -lambda_i x_j (torch-sla summary page, "Experimental
+results": 10^6 DOF, 1000 CG iterations; "Methodology" 2 for the adjoint).
+
+value      = CG iterations per second over all ranks (2000 per step per rank),
+             inputs resident in HBM, L2 flushed between steps, CUDA events.
+e2e        = the same metric through the public autograd API (CSR.solve +
+             backward) with the step's inputs copied from pinned host memory
+             and the loss read back every step.
+roofline   = the persistent CG kernel: algorithmic bytes per launch (1000
+             iterations x the per-iteration traffic of a two-pass fused PCG:
+             one sweep of A plus 11 vector passes) / its CUDA-event duration.
+cpu_baseline = the CPU oracle (single thread) on a bounded sample of the step.
+
+Multi-GPU (torchrun): every rank solves its own independent system (replicas;
+the single system is not partitioned), time = max over ranks.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CG iter/s & fwd+adjoint solve ms; SpMV/CG HBM GB/s vs B200 peak (1 GPU)"
+UNIT = "CG iterations/s"
+N_GRID, ITERS = 1024, 1000
+FALLBACK_HBM_GBS = 6650.0
+
+
+def per_iteration_bytes(n: int, nnz: int, vbytes: int) -> int:
+    """Two-pass fused PCG: A once ((vbytes + 4) nnz + 4 (n + 1)) + 11 vector passes."""
+    return (vbytes + 4) * nnz + 4 * (n + 1) + 11 * vbytes * n
+
+
+def grad_bytes(n: int, nnz: int, vbytes: int) -> int:
+    """Value gradient: colind + gradient per entry, lambda, x and rowptr per row."""
+    return (4 + vbytes) * nnz + (2 * vbytes + 4) * n
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "differentiable_sparse_linear_csr_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_key}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    if not m or not d or d.group(1) != source_digest():
+        return None
+    return float(m.group(1))
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+_WORKLOAD = {}
+
+
+def oracle_sample(dtype_name: str, k_iters: int):
+    """Oracle on a bounded sample of the step: k forward + k adjoint iterations + gradient."""
+    import numpy as np
+    from oracle import oracle as O
+    from differentiable_sparse_linear_csr_b200 import workloads as W
+    if "c2" not in _WORKLOAD:
+        _WORKLOAD["c2"] = W.c2_poisson1024(N=N_GRID, iters=ITERS)
+    w = _WORKLOAD["c2"]
+    npdt = np.float64 if dtype_name == "f64" else np.float32
+    v, b, xs = w.values[0].astype(npdt), w.b[0].astype(npdt), w.xstar[0].astype(npdt)
+    O.build()
+    t0 = time.perf_counter()
+    x, _ = O.pcg(w.rowptr, w.colind, v, b, fixed_iters=k_iters)
+    lam, _ = O.cg_adjoint(w.rowptr, w.colind, v, (x - xs).astype(npdt), fixed_iters=k_iters)
+    O.grad_values(w.rowptr, w.colind, lam, x)
+    dt = time.perf_counter() - t0
+    return 2 * k_iters / dt, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    k = args.ref_iters
+    for _ in range(args.warmup):
+        oracle_sample(args.dtype, k)
+    total_it, total_t = 0, 0.0
+    for _ in range(args.steps):
+        _, dt = oracle_sample(args.dtype, k)
+        total_it += 2 * k
+        total_t += dt
+    v = total_it / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+            "config": workload_config(args),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {k} forward + {k} adjoint PCG iterations + "
+                                       "value gradient of the 1024x1024 Poisson system"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(args):
+    n = N_GRID * N_GRID
+    return {"workload": f"2-D 5-point Dirichlet Poisson {N_GRID}x{N_GRID}: fixed {ITERS} forward + "
+                        f"{ITERS} adjoint Jacobi-PCG iterations + sparse value gradient",
+            "n": n, "nnz": 5 * n - 4 * N_GRID, "batch": 1, "value_dtype": args.dtype,
+            "l2": "flushed between steps (write of a 256 MiB buffer)",
+            "parallelism": f"replicas x{int(os.environ.get('WORLD_SIZE', '1'))}"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sla", choices=["sla", "reference"])
+    ap.add_argument("--dtype", default="f64", choices=["f64", "f32"])
+    ap.add_argument("--ref-iters", type=int, default=40)
+    ap.add_argument("--cpu-iters", type=int, default=300)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--strategy", type=int, default=0)
+    ap.add_argument("--iters", type=int, default=ITERS,
+                    help="iterations per solve; only for short profiler captures")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import differentiable_sparse_linear_csr_b200 as sla
+    from differentiable_sparse_linear_csr_b200 import _lib as L
+    from differentiable_sparse_linear_csr_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    dt = torch.float64 if args.dtype == "f64" else torch.float32
+    vbytes = 8 if args.dtype == "f64" else 4
+    w = W.c2_poisson1024(seed=2 + rank, N=N_GRID, iters=ITERS)
+    n, nnz = w.n, w.nnz
+    A = sla.CSR(torch.from_numpy(w.rowptr).to(dev), torch.from_numpy(w.colind).to(dev),
+                dtype=dt, symmetric=True)
+    vals = torch.from_numpy(w.values).to(dev, dt).contiguous()
+    b = torch.from_numpy(w.b).to(dev, dt).contiguous()
+    xs = torch.from_numpy(w.xstar).to(dev, dt).contiguous()
+    x = torch.empty(1, n, dtype=dt, device=dev)
+    g = torch.empty(1, n, dtype=dt, device=dev)
+    lam = torch.empty(1, n, dtype=dt, device=dev)
+    G = torch.empty(1, nnz, dtype=dt, device=dev)
+    info = [torch.empty(1, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    cinfo = L.make_info(*info)
+    ws = torch.empty(L.sla_workspace_bytes(A.handle, L.SLA_OP_ADJOINT), dtype=torch.uint8, device=dev)
+    iters = args.iters
+    opts = L.make_opts(fixed_iters=iters, strategy=args.strategy)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        L.sla_cg_solve(A.handle, vals, b, x, opts, cinfo, ws)
+        if e: e[1].record(stream)
+        torch.sub(x, xs, out=g)                       # dL/dx of L = 0.5 ||x - x*||^2
+        if e: e[2].record(stream)
+        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, cinfo, ws)
+        if e: e[3].record(stream)
+        L.sla_grad_values(A.handle, lam, x, G, 0)
+        if e: e[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if rank == 0 else None
+    events = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()                                  # L2 flush, outside the step's events
+        step(events[k])
+    torch.cuda.synchronize()
+    clock_info = clocks.stop() if clocks else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[4]) for e in events]
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
+    adj_ms = [e[2].elapsed_time(e[3]) for e in events]
+    grad_ms = [e[3].elapsed_time(e[4]) for e in events]
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+    iters_done = 2 * iters * args.steps * world
+    value = iters_done / (total_ms / 1000.0)
+
+    # ---- end to end through the public API, host buffers, loss read back
+    e2e = None
+    if not args.no_e2e:
+        vh = torch.from_numpy(w.values).to(dt).pin_memory()
+        bh = torch.from_numpy(w.b).to(dt).pin_memory()
+        xh = torch.from_numpy(w.xstar).to(dt).pin_memory()
+        vd = torch.empty_like(vals)
+        bd = torch.empty_like(b)
+        xd = torch.empty_like(xs)
+
+        def e2e_step():
+            vd.copy_(vh, non_blocking=True)
+            bd.copy_(bh, non_blocking=True)
+            xd.copy_(xh, non_blocking=True)
+            vv = vd.requires_grad_(True)
+            xx = A.solve(vv, bd, fixed_iters=iters, strategy=args.strategy)
+            loss = 0.5 * ((xx - xd) ** 2).sum()
+            loss.backward()
+            vv.grad = None
+            vd.requires_grad_(False)
+            return loss.item()
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e2e_ms = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms += e0.elapsed_time(e1)
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = {"value": iters_done / (float(t.item()) / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": int(vh.numel() * vh.element_size() + bh.numel() * bh.element_size()
+                                         + xh.numel() * xh.element_size()),
+               "d2h_bytes_per_step": 8}
+
+    if rank == 0:
+        peak, peak_kind = measured_hbm_peak()
+        it_bytes = per_iteration_bytes(n, nnz, vbytes)
+        cg_launch_ms = statistics.mean(fwd_ms + adj_ms)
+        achieved = iters * it_bytes / (cg_launch_ms / 1000.0) / 1e9
+        traffic = profile_traffic(f"cg_grid_kernel_c2_{args.dtype}")
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                "kernel": "cg_grid_kernel (persistent PCG, one launch per solve, %s)"
+                          % ("x, r, M^-1 on chip" if A.props.grid_onchip else "vectors in HBM"),
+                "algorithmic_bytes_per_launch": iters * it_bytes,
+                "launch_ms": cg_launch_ms}
+        gb = grad_bytes(n, nnz, vbytes)
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v_cpu, t_cpu = oracle_sample(args.dtype, args.cpu_iters)
+            cpu = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": f"{args.cpu_iters} forward + {args.cpu_iters} adjoint PCG iterations + "
+                             f"value gradient of the same system, single-threaded C ({t_cpu:.1f} s)"}
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+                "config": workload_config(args),
+                "fwd_adj_grad_ms": statistics.mean(step_ms),
+                "forward_ms": statistics.mean(fwd_ms), "adjoint_ms": statistics.mean(adj_ms),
+                "grad_ms": statistics.mean(grad_ms),
+                "grad_gbs": gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 3 * args.steps,
+                "clocks": clock_info}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

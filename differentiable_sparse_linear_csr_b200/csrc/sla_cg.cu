@@ -55,6 +55,8 @@ struct CgArgs {
 };
 
 // ------------------------------------------------------------ helpers ----
+constexpr int kMaxLocalTiles = 128;   // tiles one block of the grid kernel may own
+
 template <typename T>
 __device__ __forceinline__ void finalize(const CgArgs<T> &a, int s, int status, int iters,
                                          double relres, bool count_down) {
@@ -65,40 +67,84 @@ __device__ __forceinline__ void finalize(const CgArgs<T> &a, int s, int status, 
     if (count_down) atomicSub(a.sync + 3, 1u);
 }
 
-// Sum of a system's tile partials, in tile order per lane and a fixed xor tree
-// across lanes: the same value in every block.  NV arrays at once; results in
-// out[0..NV) for all threads of the block.
-template <int NV>
-__device__ __forceinline__ void system_sums(const double *const (&arr)[NV], int ntiles,
-                                            double *out) {
-    __syncthreads();
-    if (threadIdx.x < 32) {
+// Deterministic block sum of NV doubles per thread (fixed xor tree in each warp,
+// then warp totals in warp order); every thread gets the sums.  red >= 33*NV.
+template <int NT, int NV>
+__device__ __forceinline__ void block_sums(double (&v)[NV], double *red) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            double acc = 0.0;
-            for (int j = threadIdx.x; j < ntiles; j += 32) acc += __ldcg(arr[v] + j);
-            acc = warp_sum(acc);
-            if (threadIdx.x == 0) out[v] = acc;
+    for (int k = 0; k < NV; ++k) {
+        v[k] = warp_sum(v[k]);
+        if (lane == 0) red[k * 33 + warp] = v[k];
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            double s = lane < NW ? red[k * 33 + lane] : 0.0;
+            s = warp_sum(s);
+            if (lane == 0) red[k * 33 + 32] = s;
         }
     }
     __syncthreads();
+#pragma unroll
+    for (int k = 0; k < NV; ++k) v[k] = red[k * 33 + 32];
+    __syncthreads();
 }
 
-__device__ __forceinline__ int read_state_uniform(const int *state, int s, int *sh) {
-    __syncthreads();
-    if (threadIdx.x == 0) *sh = __ldcg(state + s);
-    __syncthreads();
-    return *sh;
+// Sum over a system's tile partials.  Thread t takes partials t, t+NT, ... in
+// order and the block tree combines them, so every block computes the same
+// value; all partials are fetched in one round of parallel loads.
+template <int NT, int NV>
+__device__ __forceinline__ void system_sums(const double *const (&arr)[NV], int ntiles,
+                                            double (&out)[NV], double *red) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        double acc = 0.0;
+        for (int j = threadIdx.x; j < ntiles; j += NT) acc += __ldcg(arr[k] + j);
+        out[k] = acc;
+    }
+    block_sums<NT, NV>(out, red);
 }
 
-// Device-wide barrier that also reports, block-uniformly, the number of
-// systems still active as seen after the barrier.
-__device__ __forceinline__ bool barrier_and_watch(unsigned *sync, long long timeout_ns,
-                                                  int *flag, unsigned *active) {
-    const bool ok = grid_barrier(sync, gridDim.x, timeout_ns, flag);
-    if (threadIdx.x == 0) *active = ld_acquire_u32(sync + 3);
+// Device-wide barrier on a monotonically increasing arrival counter: the k-th
+// barrier of the launch completes when the counter reaches k * gridDim.x, a
+// target every block knows, so arrival is a single fire-and-forget add and the
+// wait is one polling load.  sync[0] counts, sync[2] is the error flag.  Each
+// wait is bounded by timeout_ns of %globaltimer (checked on the first poll and
+// every 8th after); a block that gives up raises the flag and blocks that see
+// it give up too.  If `watch` is given, thread 0 also reads it after the
+// barrier and *watched holds the value for the whole block.
+__device__ __forceinline__ bool grid_sync(unsigned *sync, unsigned &target, long long timeout_ns,
+                                          int *flag, const unsigned *watch = nullptr,
+                                          unsigned *watched = nullptr) {
     __syncthreads();
-    return ok;
+    target += gridDim.x;
+    if (threadIdx.x == 0) {
+        unsigned *count = sync, *err = sync + 2;
+        int ok = 1;
+        __threadfence();
+        atomicAdd(count, 1u);
+        const unsigned long long t0 = global_timer_ns();
+        unsigned spins = 0;
+        while ((int)(ld_acquire_u32(count) - target) < 0) {
+            if ((spins++ & 7u) == 0) {
+                if (ld_acquire_u32(err) != 0) { ok = 0; break; }
+                if ((long long)(global_timer_ns() - t0) > timeout_ns) {
+                    atomicExch(err, 1u);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        if (ok && ld_acquire_u32(err) != 0) ok = 0;
+        __threadfence();
+        if (watch) *watched = ld_acquire_u32(watch);
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
 }
 
 template <typename T>
@@ -114,80 +160,100 @@ __device__ void give_up(const CgArgs<T> &a) {
 }
 
 // ------------------------------------------------------- grid kernel ----
-template <typename T, int LANES>
-__global__ void __launch_bounds__(kCgThreads)
+// Every block owns the tiles blockIdx.x + lt * gridDim.x (lt = 0, 1, ...) for
+// the whole solve and takes the decisions (breakdown, stop, alpha, beta) for
+// them itself from the shared partials; ONCHIP keeps x, r and M^-1 of its one
+// tile in shared memory and q in registers (RPT rows a thread), so only A and
+// p travel through L2/HBM each iteration.
+template <typename T, int LANES, bool ONCHIP, int RPT, int NT>
+__global__ void __launch_bounds__(NT, ONCHIP ? 1 : 2)
 cg_grid_kernel(CgArgs<T> a) {
-    __shared__ double red[72];
-    __shared__ double bc[4];
-    __shared__ int flag, st_sh;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ double red[4 * 33];
+    __shared__ double l_rho[kMaxLocalTiles], l_nb[kMaxLocalTiles], l_rr[kMaxLocalTiles],
+        l_alpha[kMaxLocalTiles];
+    __shared__ int l_state[kMaxLocalTiles];
+    __shared__ int flag;
     __shared__ unsigned active;
-    constexpr int NSUB = kCgThreads / LANES;
+    constexpr int NSUB = NT / LANES;
     const int tid = threadIdx.x, sub = tid / LANES, lane = tid % LANES;
     const int ntot = a.B * a.ntiles;
+    const int G = gridDim.x;
+    const int nlt = blockIdx.x < ntot ? (ntot - blockIdx.x + G - 1) / G : 0;
+    // With one system spread over every block, each block sees every decision;
+    // otherwise the count of active systems decides when the loop ends.
+    const bool local_end = (a.B == 1 && a.ntiles >= G);
     double *P0 = a.part, *P1 = P0 + ntot, *P2 = P1 + ntot, *P3 = P2 + ntot;
-    double *rho = a.sysd, *nbv = a.sysd + 2 * a.B, *rrv = a.sysd + 3 * a.B;
     const int n = a.n;
+    unsigned target = 0;
+    T qreg[ONCHIP ? RPT : 1];
+    T *xs_ = reinterpret_cast<T *>(smem_raw);     // ONCHIP: [tile_rows] each
+    T *rs_ = xs_ + (ONCHIP ? a.tile_rows : 0);
+    T *ds_ = rs_ + (ONCHIP ? a.tile_rows : 0);
 
     if (blockIdx.x == 0 && tid == 0) a.sync[3] = (unsigned)a.B;
 
     // ---- init: r = b - A x0 (or b), z = M^-1 r, p = z; partials of b.b, r.z, r.r
-    for (int tile = blockIdx.x; tile < ntot; tile += gridDim.x) {
+    for (int lt = 0; lt < nlt; ++lt) {
+        const int tile = blockIdx.x + lt * G;
         const int s = tile / a.ntiles, tt = tile % a.ntiles;
         const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
         const T *vs = a.vals + (int64_t)s * a.nnz;
         const T *bs = a.b + (int64_t)s * n;
-        T *xs = a.x + (int64_t)s * n, *rs = a.r + (int64_t)s * n, *ps = a.p + (int64_t)s * n;
-        T *qs = a.q + (int64_t)s * n, *ds = a.d + (int64_t)s * n;
+        T *xg = a.x + (int64_t)s * n, *pg = a.p + (int64_t)s * n, *qg = a.q + (int64_t)s * n;
         if (a.x0_given) {
             for (int i = r0 + sub; i < r1; i += NSUB) {
-                const T v = row_dot<T, LANES>(a.rowptr, a.colind, vs, xs, i, lane);
-                if (lane == 0) qs[i] = v;
+                const T v = row_dot<T, LANES>(a.rowptr, a.colind, vs, xg, i, lane);
+                if (lane == 0) qg[i] = v;
             }
             __syncthreads();
         }
-        double lbb = 0.0, lrho = 0.0, lrr = 0.0, lbad = 0.0;
-        for (int i = r0 + tid; i < r1; i += kCgThreads) {
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};   // b.b, r.z, r.r, bad diagonals
+        for (int i = r0 + tid; i < r1; i += NT) {
             const T bi = bs[i];
-            T ri;
-            if (a.x0_given) {
-                ri = bi - qs[i];
-            } else {
-                ri = bi;
-                xs[i] = T(0);
-            }
+            const T xi = a.x0_given ? xg[i] : T(0);
+            const T ri = a.x0_given ? bi - qg[i] : bi;
             T di = T(1);
             if (a.precond) {
                 const int dp = __ldg(a.diagpos + i);
                 const T dv = dp >= 0 ? __ldg(vs + dp) : T(0);
-                if (!(dv > T(0))) lbad += 1.0;
+                if (!(dv > T(0))) acc[3] += 1.0;
                 di = T(1) / dv;
             }
             const T zi = di * ri;
-            rs[i] = ri;
-            ps[i] = zi;
-            ds[i] = di;
-            lbb += (double)bi * (double)bi;
-            lrho += (double)ri * (double)zi;
-            lrr += (double)ri * (double)ri;
+            pg[i] = zi;
+            if constexpr (ONCHIP) {
+                xs_[i - r0] = xi;
+                rs_[i - r0] = ri;
+                ds_[i - r0] = di;
+            } else {
+                if (!a.x0_given) xg[i] = T(0);
+                a.r[(int64_t)s * n + i] = ri;
+                a.d[(int64_t)s * n + i] = di;
+            }
+            acc[0] += (double)bi * (double)bi;
+            acc[1] += (double)ri * (double)zi;
+            acc[2] += (double)ri * (double)ri;
         }
-        block_sum2<kCgThreads>(lbb, lrho, red);
-        block_sum2<kCgThreads>(lrr, lbad, red);
+        block_sums<NT, 4>(acc, red);
         if (tid == 0) {
-            P0[tile] = lbb;
-            P1[tile] = lrho;
-            P2[tile] = lrr;
-            P3[tile] = lbad;
+            P0[tile] = acc[0];
+            P1[tile] = acc[1];
+            P2[tile] = acc[2];
+            P3[tile] = acc[3];
         }
     }
-    if (!grid_barrier(a.sync, gridDim.x, a.timeout_ns, &flag)) { give_up(a); return; }
+    if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
 
-    // ---- initial decisions, made identically by every block holding a tile
-    for (int tile = blockIdx.x; tile < ntot; tile += gridDim.x) {
+    // ---- initial decisions, taken identically by every block holding a tile
+    for (int lt = 0; lt < nlt; ++lt) {
+        const int tile = blockIdx.x + lt * G;
         const int s = tile / a.ntiles, tt = tile % a.ntiles;
         const int off = s * a.ntiles;
         const double *const arr[4] = {P0 + off, P1 + off, P2 + off, P3 + off};
-        system_sums<4>(arr, a.ntiles, bc);
-        const double bb = bc[0], rho0 = bc[1], rr = bc[2], bad = bc[3];
+        double sum[4];
+        system_sums<NT, 4>(arr, a.ntiles, sum, red);
+        const double bb = sum[0], rho0 = sum[1], rr = sum[2], bad = sum[3];
         const double nb = sqrt(bb);
         const double tol = fmax(a.rtol * nb, a.atol);
         int st = kActive;
@@ -197,110 +263,191 @@ cg_grid_kernel(CgArgs<T> a) {
         else if (a.precond && bad > 0.0) { st = SLA_BREAKDOWN; relres = sqrt(rr) / nb; }
         else if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; relres = sqrt(rr) / nb; }
         else if (rr == 0.0) st = SLA_CONVERGED;
-        if (nb == 0.0 && a.x0_given) {
+        if (nb == 0.0) {
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
-            T *xs = a.x + (int64_t)s * n;
-            for (int i = r0 + tid; i < r1; i += kCgThreads) xs[i] = T(0);
+            for (int i = r0 + tid; i < r1; i += NT) {
+                if constexpr (ONCHIP) xs_[i - r0] = T(0);
+                else a.x[(int64_t)s * n + i] = T(0);
+            }
         }
-        if (tt == 0 && tid == 0) {
-            rho[s] = rho0;
-            nbv[s] = nb;
-            rrv[s] = rr;
-            if (st == kActive) a.state[s] = kActive;
-            else finalize(a, s, st, 0, relres, true);
+        if (tid == 0) {
+            l_state[lt] = st;
+            l_rho[lt] = rho0;
+            l_nb[lt] = nb;
+            l_rr[lt] = rr;
+            if (tt == 0) {
+                if (st == kActive) a.state[s] = kActive;
+                else finalize(a, s, st, 0, relres, true);
+            }
         }
     }
-    if (!barrier_and_watch(a.sync, a.timeout_ns, &flag, &active)) { give_up(a); return; }
+    __syncthreads();
+    bool more;
+    if (local_end) {
+        more = nlt > 0 && l_state[0] == kActive;
+    } else {
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag, a.sync + 3, &active)) { give_up(a); return; }
+        more = active != 0;
+    }
 
     int k = 0;
-    while (active != 0) {
+    while (more) {
         // ---- phase A: q = A p and the partials of p.q
-        for (int tile = blockIdx.x; tile < ntot; tile += gridDim.x) {
+        for (int lt = 0; lt < nlt; ++lt) {
+            if (l_state[lt] != kActive) continue;
+            const int tile = blockIdx.x + lt * G;
             const int s = tile / a.ntiles, tt = tile % a.ntiles;
-            if (read_state_uniform(a.state, s, &st_sh) != kActive) continue;
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
             const T *vs = a.vals + (int64_t)s * a.nnz;
-            const T *ps = a.p + (int64_t)s * n;
-            T *qs = a.q + (int64_t)s * n;
-            double ls = 0.0;
-            for (int i = r0 + sub; i < r1; i += NSUB) {
-                const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, ps, i, lane);
-                if (lane == 0) {
-                    qs[i] = qi;
-                    ls += (double)ps[i] * (double)qi;
+            const T *pg = a.p + (int64_t)s * n;
+            double acc[1] = {0.0};
+            if constexpr (ONCHIP) {
+#pragma unroll
+                for (int j = 0; j < RPT; ++j) {
+                    const int i = r0 + tid + j * NT;
+                    if (i < r1) {
+                        const T qi = row_dot<T, 1>(a.rowptr, a.colind, vs, pg, i, 0);
+                        qreg[j] = qi;
+                        acc[0] += (double)pg[i] * (double)qi;
+                    }
+                }
+            } else {
+                T *qg = a.q + (int64_t)s * n;
+                for (int i = r0 + sub; i < r1; i += NSUB) {
+                    const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, pg, i, lane);
+                    if (lane == 0) {
+                        qg[i] = qi;
+                        acc[0] += (double)pg[i] * (double)qi;
+                    }
                 }
             }
-            ls = block_sum<kCgThreads>(ls, red);
-            if (tid == 0) P0[tile] = ls;
+            block_sums<NT, 1>(acc, red);
+            if (tid == 0) P0[tile] = acc[0];
         }
-        if (!grid_barrier(a.sync, gridDim.x, a.timeout_ns, &flag)) { give_up(a); return; }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
         ++k;
 
-        // ---- phase B: alpha; x += alpha p; r -= alpha q; partials of r.z, r.r
-        for (int tile = blockIdx.x; tile < ntot; tile += gridDim.x) {
+        // ---- phase B: alpha; r -= alpha q; partials of r.z and r.r
+        for (int lt = 0; lt < nlt; ++lt) {
+            if (l_state[lt] != kActive) continue;
+            const int tile = blockIdx.x + lt * G;
             const int s = tile / a.ntiles, tt = tile % a.ntiles;
-            if (read_state_uniform(a.state, s, &st_sh) != kActive) continue;
             const double *const arr[1] = {P0 + s * a.ntiles};
-            system_sums<1>(arr, a.ntiles, bc);
-            const double sigma = bc[0];
+            double sg[1];
+            system_sums<NT, 1>(arr, a.ntiles, sg, red);
+            const double sigma = sg[0];
             if (!isfinite(sigma) || !(sigma > 0.0)) {
-                if (tt == 0 && tid == 0)
-                    finalize(a, s, isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE, k - 1,
-                             sqrt(rrv[s]) / nbv[s], true);
+                const int st = isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE;
+                if (tid == 0) {
+                    l_state[lt] = st;
+                    if (tt == 0) finalize(a, s, st, k - 1, sqrt(l_rr[lt]) / l_nb[lt], true);
+                }
+                __syncthreads();
                 continue;
             }
-            const T al = (T)(__ldcg(rho + ((k - 1) & 1) * a.B + s) / sigma);
+            const double alpha = l_rho[lt] / sigma;
+            const T al = (T)alpha;
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
-            T *xs = a.x + (int64_t)s * n, *rs = a.r + (int64_t)s * n;
-            const T *ps = a.p + (int64_t)s * n, *qs = a.q + (int64_t)s * n, *ds = a.d + (int64_t)s * n;
-            double lrho = 0.0, lrr = 0.0;
-            for (int i = r0 + tid; i < r1; i += kCgThreads) {
-                const T pi = ps[i];
-                xs[i] = xs[i] + al * pi;
-                const T ri = rs[i] - al * qs[i];
-                rs[i] = ri;
-                const T zi = ds[i] * ri;
-                lrho += (double)ri * (double)zi;
-                lrr += (double)ri * (double)ri;
+            double acc[2] = {0.0, 0.0};
+            if constexpr (ONCHIP) {
+#pragma unroll
+                for (int j = 0; j < RPT; ++j) {
+                    const int i = r0 + tid + j * NT;
+                    if (i < r1) {
+                        const T ri = rs_[i - r0] - al * qreg[j];
+                        rs_[i - r0] = ri;
+                        const T zi = ds_[i - r0] * ri;
+                        acc[0] += (double)ri * (double)zi;
+                        acc[1] += (double)ri * (double)ri;
+                    }
+                }
+            } else {
+                T *rg = a.r + (int64_t)s * n;
+                const T *qg = a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                for (int i = r0 + tid; i < r1; i += NT) {
+                    const T ri = rg[i] - al * qg[i];
+                    rg[i] = ri;
+                    const T zi = dg[i] * ri;
+                    acc[0] += (double)ri * (double)zi;
+                    acc[1] += (double)ri * (double)ri;
+                }
             }
-            block_sum2<kCgThreads>(lrho, lrr, red);
+            block_sums<NT, 2>(acc, red);
             if (tid == 0) {
-                P1[tile] = lrho;
-                P2[tile] = lrr;
+                P1[tile] = acc[0];
+                P2[tile] = acc[1];
+                l_alpha[lt] = alpha;
             }
         }
-        if (!grid_barrier(a.sync, gridDim.x, a.timeout_ns, &flag)) { give_up(a); return; }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
 
-        // ---- phase C: stopping test; beta; p = z + beta p
-        for (int tile = blockIdx.x; tile < ntot; tile += gridDim.x) {
+        // ---- phase C: x += alpha p; stopping test; beta; p = z + beta p
+        for (int lt = 0; lt < nlt; ++lt) {
+            if (l_state[lt] != kActive) continue;
+            const int tile = blockIdx.x + lt * G;
             const int s = tile / a.ntiles, tt = tile % a.ntiles;
-            if (read_state_uniform(a.state, s, &st_sh) != kActive) continue;
             const double *const arr[2] = {P1 + s * a.ntiles, P2 + s * a.ntiles};
-            system_sums<2>(arr, a.ntiles, bc);
-            const double rho_new = bc[0], rr = bc[1];
-            const double nb = __ldcg(nbv + s);
+            double sum[2];
+            system_sums<NT, 2>(arr, a.ntiles, sum, red);
+            const double rho_new = sum[0], rr = sum[1];
+            const double nb = l_nb[lt];
             const double tol = fmax(a.rtol * nb, a.atol);
             int st = kActive;
             if (!isfinite(rr)) st = SLA_NONFINITE;
             else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
             else if (rr == 0.0) st = SLA_CONVERGED;
             else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
-            if (st != kActive) {
-                if (tt == 0 && tid == 0) finalize(a, s, st, k, sqrt(rr) / nb, true);
-                continue;
-            }
-            const double rho_old = __ldcg(rho + ((k - 1) & 1) * a.B + s);
-            const T bt = (T)(rho_new / rho_old);
+            const T al = (T)l_alpha[lt];
+            const T bt = (T)(rho_new / l_rho[lt]);
+            const bool go_on = st == kActive;
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
-            const T *rs = a.r + (int64_t)s * n, *ds = a.d + (int64_t)s * n;
-            T *ps = a.p + (int64_t)s * n;
-            for (int i = r0 + tid; i < r1; i += kCgThreads) ps[i] = ds[i] * rs[i] + bt * ps[i];
-            if (tt == 0 && tid == 0) {
-                rho[(k & 1) * a.B + s] = rho_new;
-                rrv[s] = rr;
+            T *pg = a.p + (int64_t)s * n;
+            if constexpr (ONCHIP) {
+#pragma unroll
+                for (int j = 0; j < RPT; ++j) {
+                    const int i = r0 + tid + j * NT;
+                    if (i < r1) {
+                        const T pi = pg[i];
+                        xs_[i - r0] = xs_[i - r0] + al * pi;
+                        if (go_on) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pi;
+                    }
+                }
+            } else {
+                T *xg = a.x + (int64_t)s * n;
+                const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                for (int i = r0 + tid; i < r1; i += NT) {
+                    const T pi = pg[i];
+                    xg[i] = xg[i] + al * pi;
+                    if (go_on) pg[i] = dg[i] * rg[i] + bt * pi;
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                if (go_on) {
+                    l_rho[lt] = rho_new;
+                    l_rr[lt] = rr;
+                } else {
+                    l_state[lt] = st;
+                    if (tt == 0) finalize(a, s, st, k, sqrt(rr) / nb, true);
+                }
             }
         }
-        if (!barrier_and_watch(a.sync, a.timeout_ns, &flag, &active)) { give_up(a); return; }
+        if (local_end) {
+            if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
+            more = l_state[0] == kActive;
+        } else {
+            if (!grid_sync(a.sync, target, a.timeout_ns, &flag, a.sync + 3, &active)) { give_up(a); return; }
+            more = active != 0;
+        }
+    }
+    if constexpr (ONCHIP) {
+        for (int lt = 0; lt < nlt; ++lt) {
+            const int tile = blockIdx.x + lt * G;
+            const int s = tile / a.ntiles, tt = tile % a.ntiles;
+            const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
+            T *xg = a.x + (int64_t)s * n;
+            for (int i = r0 + tid; i < r1; i += NT) xg[i] = xs_[i - r0];
+        }
     }
 }
 
@@ -426,8 +573,16 @@ __global__ void info_fill_kernel(int B, int32_t *iters, double *relres, int32_t 
 }
 
 // ----------------------------------------------------------- host side ----
+constexpr int kOnchipThreads = 1024;
+
 template <typename T, int L>
-static const void *grid_fn() { return reinterpret_cast<const void *>(&cg_grid_kernel<T, L>); }
+static const void *grid_fn() {
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, L, false, 1, kCgThreads>);
+}
+template <typename T, int RPT>
+static const void *onchip_fn() {
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads>);
+}
 template <typename T, int L>
 static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L>); }
 
@@ -440,6 +595,29 @@ static const void *pick_fn(bool grid, sla_dtype dt, int lanes) {
         return SLA_OK;
     });
     return f;
+}
+
+static const void *pick_onchip(sla_dtype dt, int rpt) {
+    if (dt == SLA_F64) {
+        if (rpt <= 4) return onchip_fn<double, 4>();
+        if (rpt <= 8) return onchip_fn<double, 8>();
+        return onchip_fn<double, 16>();
+    }
+    if (rpt <= 4) return onchip_fn<float, 4>();
+    if (rpt <= 8) return onchip_fn<float, 8>();
+    return onchip_fn<float, 16>();
+}
+
+// Tile layout: tiles never straddle systems, and B * ntiles <= blocks whenever
+// B <= blocks, so that each block owns at most one tile in the common case.
+static void layout(Csr *h, int blocks, int32_t *tile_rows, int32_t *ntiles) {
+    const int n = h->n_rows, B = h->batch;
+    int nt = blocks / B;
+    if (nt < 1) nt = 1;
+    int64_t tr = n > 0 ? ((int64_t)n + nt - 1) / nt : 1;
+    if (tr > 32) tr = (tr + 31) / 32 * 32;
+    *tile_rows = (int32_t)tr;
+    *ntiles = n > 0 ? (int32_t)(((int64_t)n + tr - 1) / tr) : 1;
 }
 
 sla_status cg_configure(Csr *h) {
@@ -455,25 +633,49 @@ sla_status cg_configure(Csr *h) {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             optin - 2048));
     }
-    int per_sm = 0;
-    SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &per_sm, pick_fn(true, h->dtype, h->lanes), kCgThreads, 0));
-    int want = 2;
-    if (const char *e = getenv("SLA_GRID_BLOCKS_PER_SM")) want = atoi(e);
-    if (want < 1) want = 1;
-    per_sm = per_sm < want ? per_sm : want;
-    if (per_sm < 1) {
-        set_error("cg_configure: persistent kernel cannot be resident");
-        return SLA_ERR_CUDA;
+    // On-chip variant: one 1024-thread block per SM, x, r, M^-1 of the block's
+    // rows in shared memory, at most 16 rows a thread.
+    h->onchip = false;
+    const char *oc = getenv("SLA_GRID_ONCHIP");
+    if (h->lanes == 1 && n > 0 && !(oc && oc[0] == '0')) {
+        int32_t tr = 0, nt = 0;
+        layout(h, h->num_sms, &tr, &nt);
+        const int rpt = (tr + kOnchipThreads - 1) / kOnchipThreads;
+        const size_t smem = 3 * (size_t)tr * ts;
+        if ((int64_t)h->batch * nt <= h->num_sms && rpt <= 16 && smem + 16384 <= (size_t)optin) {
+            const void *f = pick_onchip(h->dtype, rpt);
+            SLA_CHECK_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                optin - 16384));
+            int per_sm = 0;
+            SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kOnchipThreads, smem));
+            if (per_sm >= 1) {
+                h->onchip = true;
+                h->onchip_rpt = rpt;
+                h->grid_smem = smem;
+                h->grid_threads = kOnchipThreads;
+                h->grid_blocks = h->num_sms;
+                h->tile_rows = tr;
+                h->ntiles = nt;
+            }
+        }
     }
-    h->grid_blocks = per_sm * h->num_sms;
-    const int B = h->batch;
-    int ntiles = h->grid_blocks / B;
-    if (ntiles < 1) ntiles = 1;
-    int64_t tr = n > 0 ? ((int64_t)n + ntiles - 1) / ntiles : 1;
-    if (tr > 32) tr = (tr + 31) / 32 * 32;
-    h->tile_rows = (int32_t)tr;
-    h->ntiles = n > 0 ? (int32_t)(((int64_t)n + tr - 1) / tr) : 1;
+    if (!h->onchip) {
+        int per_sm = 0;
+        SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, pick_fn(true, h->dtype, h->lanes), kCgThreads, 0));
+        int want = 2;
+        if (const char *e = getenv("SLA_GRID_BLOCKS_PER_SM")) want = atoi(e);
+        if (want < 1) want = 1;
+        per_sm = per_sm < want ? per_sm : want;
+        if (per_sm < 1) {
+            set_error("cg_configure: persistent kernel cannot be resident");
+            return SLA_ERR_CUDA;
+        }
+        h->grid_blocks = per_sm * h->num_sms;
+        h->grid_threads = kCgThreads;
+        h->grid_smem = 0;
+        layout(h, h->grid_blocks, &h->tile_rows, &h->ntiles);
+    }
     return SLA_OK;
 }
 
@@ -530,11 +732,19 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
         use_grid = !h->block_fits;
     }
     if (use_grid) {
+        const int ntot = a.B * a.ntiles;
+        const int nlt = (ntot + h->grid_blocks - 1) / h->grid_blocks;
+        if (nlt > kMaxLocalTiles) {
+            set_error("sla_cg: %d systems of %d rows need %d tiles a block (limit %d); "
+                      "use smaller batches", a.B, a.n, nlt, kMaxLocalTiles);
+            return SLA_ERR_UNSUPPORTED;
+        }
         SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
         void *args[] = {&a};
-        SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(pick_fn(true, h->dtype, h->lanes),
-                                                   dim3(h->grid_blocks), dim3(kCgThreads), args,
-                                                   0, s));
+        const void *f = h->onchip ? pick_onchip(h->dtype, h->onchip_rpt)
+                                  : pick_fn(true, h->dtype, h->lanes);
+        SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(f, dim3(h->grid_blocks), dim3(h->grid_threads),
+                                                   args, h->grid_smem, s));
     } else {
         const int per = h->num_sms * 4;
         const int grid = a.B < per ? a.B : per;

@@ -92,6 +92,10 @@ struct Csr {
     int32_t tile_rows = 0;             // rows of one tile (tiles never straddle systems)
     int32_t ntiles = 0;                // tiles per system
     bool block_fits = false;           // one system fits the block-per-system solver
+    bool onchip = false;               // grid solver keeps x, r, M^-1 in shared memory
+    int32_t onchip_rpt = 0;            // rows a thread in the on-chip grid solver
+    int32_t grid_threads = 0;          // threads of a grid-solver block
+    size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
 };
 

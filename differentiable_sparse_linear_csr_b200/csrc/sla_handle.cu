@@ -305,6 +305,8 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_blocks = h->grid_blocks;
     p->block_fits = h->block_fits ? 1 : 0;
     p->has_transpose = h->has_transpose ? 1 : 0;
+    p->grid_onchip = h->onchip ? 1 : 0;
+    p->grid_tile_rows = h->tile_rows;
     return SLA_OK;
 }
 

@@ -122,6 +122,10 @@ typedef struct {
     int32_t grid_blocks;      /* persistent-grid size on this device */
     int32_t block_fits;       /* 1 if one system fits the block-per-system solver */
     int32_t has_transpose;    /* 1 once A^T's pattern is built */
+    int32_t grid_onchip;      /* 1 if the grid solver keeps x, r, M^-1 on chip (else in HBM);
+                                 the environment variable SLA_GRID_ONCHIP=0, read at
+                                 creation, turns this variant off */
+    int32_t grid_tile_rows;   /* rows of one grid-solver tile */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */

@@ -251,9 +251,12 @@ def _cases():
     yield "c4x24", w.rowptr, w.colind, w.values, w.b
 
 
-@pytest.mark.parametrize("strategy", [L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK])
+@pytest.mark.parametrize("strategy,onchip", [(L.SLA_STRATEGY_GRID, "1"), (L.SLA_STRATEGY_GRID, "0"),
+                                              (L.SLA_STRATEGY_BLOCK, "1")])
 @pytest.mark.parametrize("dtype", [torch.float64, torch.float32])
-def test_pcg_fixed_iterations_parity(strategy, dtype):
+def test_pcg_fixed_iterations_parity(strategy, onchip, dtype, monkeypatch):
+    """Both grid variants (x, r, M^-1 on chip or in HBM) and the block solver."""
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     npdt = np.float64 if dtype == torch.float64 else np.float32
     tol = TOL_X64 if dtype == torch.float64 else TOL_X32
     for name, rp, ci, v, b in _cases():
@@ -261,6 +264,8 @@ def test_pcg_fixed_iterations_parity(strategy, dtype):
         A = make(rp, ci, B=B, dtype=dtype)
         if strategy == L.SLA_STRATEGY_BLOCK and not A.props.block_fits:
             continue
+        if strategy == L.SLA_STRATEGY_GRID and onchip == "0":
+            assert A.props.grid_onchip == 0
         for k in (1, 7, 60):
             x, info = A.cg(T(v.astype(npdt)), T(b.astype(npdt)), fixed_iters=k, strategy=strategy)
             xo, io = O.pcg(rp, ci, v.astype(npdt), b.astype(npdt), fixed_iters=k)
@@ -269,9 +274,11 @@ def test_pcg_fixed_iterations_parity(strategy, dtype):
             assert max(rel_rows(H(x), xo)) < tol, (name, k)
 
 
-@pytest.mark.parametrize("strategy", [L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK])
-def test_pcg_tolerance_mode_parity(strategy):
+@pytest.mark.parametrize("strategy,onchip", [(L.SLA_STRATEGY_GRID, "1"), (L.SLA_STRATEGY_GRID, "0"),
+                                              (L.SLA_STRATEGY_BLOCK, "1")])
+def test_pcg_tolerance_mode_parity(strategy, onchip, monkeypatch):
     """Iteration counts agree within max(2, 1%); iterates agree at the oracle's count."""
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     for name, rp, ci, v, b in _cases():
         B = v.shape[0]
         A = make(rp, ci, B=B)
@@ -297,7 +304,9 @@ def test_grid_and_block_strategies_agree():
     assert np.all(np.abs(H(ig.iters) - H(ib.iters)) <= 2)
 
 
-def test_results_are_bitwise_reproducible():
+@pytest.mark.parametrize("onchip", ["1", "0"])
+def test_results_are_bitwise_reproducible(onchip, monkeypatch):
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     w = W.c1_poisson64()
     A = make(w.rowptr, w.colind)
     for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK):
@@ -447,7 +456,9 @@ def test_single_unknown_and_empty_matrix():
     assert x.shape == (2, 0) and np.all(H(info.status) == 0) and np.all(H(info.iters) == 0)
 
 
-def test_bounded_wait_times_out_without_hanging():
+@pytest.mark.parametrize("onchip", ["1", "0"])
+def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     rp, ci, v = W.poisson2d(300)
     A = make(rp, ci)
     b = T(W.normal(2, 0, 300 * 300))
