@@ -364,6 +364,7 @@ cg_grid_kernel(CgArgs<T> a) {
             } else {
                 T *rg = a.r + (int64_t)s * n;
                 const T *qg = a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+#pragma unroll 4
                 for (int i = r0 + tid; i < r1; i += NT) {
                     const T ri = rg[i] - al * qg[i];
                     rg[i] = ri;
@@ -415,6 +416,7 @@ cg_grid_kernel(CgArgs<T> a) {
             } else {
                 T *xg = a.x + (int64_t)s * n;
                 const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+#pragma unroll 4
                 for (int i = r0 + tid; i < r1; i += NT) {
                     const T pi = pg[i];
                     xg[i] = xg[i] + al * pi;
@@ -642,7 +644,8 @@ sla_status cg_configure(Csr *h) {
         layout(h, h->num_sms, &tr, &nt);
         const int rpt = (tr + kOnchipThreads - 1) / kOnchipThreads;
         const size_t smem = 3 * (size_t)tr * ts;
-        if ((int64_t)h->batch * nt <= h->num_sms && rpt <= 16 && smem + 16384 <= (size_t)optin) {
+        const int rpt_cap = h->dtype == SLA_F64 ? 8 : 16;   // beyond this the q registers spill
+        if ((int64_t)h->batch * nt <= h->num_sms && rpt <= rpt_cap && smem + 16384 <= (size_t)optin) {
             const void *f = pick_onchip(h->dtype, rpt);
             SLA_CHECK_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 optin - 16384));
