@@ -72,6 +72,8 @@ _SIGNATURES = {
     "sla_coo_workspace_bytes": ([_I32, _I32, _I64], _SZ),
     "sla_csr_from_coo": ([_I32, _I32, _I64, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "sla_csr_check": ([_I32, _I32, _I64, _P, _P, _I32, _P, _P], _I32),
+    "sla_cg_solve_noalloc": ([_I32, _I64, _P, _P, _I32, _I32, _P, _P, _P, ctypes.POINTER(sla_cg_opts),
+                              sla_cg_info, _P], _I32),
     "sla_last_error_string": ([], ctypes.c_char_p),
     "sla_version": ([], ctypes.c_char_p),
 }
@@ -225,3 +227,10 @@ def sla_csr_from_coo(n_rows, n_cols, nnz_in, row, col, batch, dtype, val, rowptr
 def sla_csr_check(n_rows, n_cols, nnz, rowptr, colind, need_diag, result, stream=None) -> None:
     _check("sla_csr_check", lib().sla_csr_check(n_rows, n_cols, nnz, _ptr(rowptr), _ptr(colind),
                                                 int(need_diag), _ptr(result), _stream(stream)))
+
+
+def sla_cg_solve_noalloc(n, nnz, rowptr, colind, batch, dtype, vals, b, x, opts, info, stream=None) -> None:
+    """Allocation-free solve: scratch in the library's static device array (no workspace)."""
+    _check("sla_cg_solve_noalloc", lib().sla_cg_solve_noalloc(
+        n, nnz, _ptr(rowptr), _ptr(colind), batch, dtype, _ptr(vals), _ptr(b), _ptr(x),
+        ctypes.byref(opts), info, _stream(stream)))

@@ -24,6 +24,7 @@
 //    shared memory (small systems, large batches): no device-wide barrier.
 #include <cmath>
 #include <cstdlib>
+#include <mutex>
 
 #include "sla_rows.cuh"
 
@@ -834,4 +835,163 @@ extern "C" sla_status sla_cg_adjoint(sla_csr_t hh, const void *vals, const void 
     clear_error();
     return cg_entry(reinterpret_cast<Csr *>(hh), vals, g, lambda, opts, info, ws, ws_bytes, stream,
                     true);
+}
+
+// ------------------------------------------------ allocation-free solve ----
+// The same persistent solver for callers that may not allocate device memory
+// while they solve: runtimes that reserve all device memory up front and hand
+// it out themselves, loops that cannot afford the device-wide synchronisation
+// that cudaMalloc and cudaFree may imply, and plugins that must not call into
+// their host application's allocator.  Its scratch (synchronisation words, partial sums, per-system
+// scalars, diagonal positions and the r, p, q, M^-1 vectors) lives in one
+// file-scope device array that every GPU loading this library keeps until the
+// process exits.  The array is shared by all calls on a device and keeps what
+// the last call left there, so this entry point clears what must start at
+// zero, and calls whose kernels overlap on the GPU race on it.
+namespace sla {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static void *g_noalloc_ptr[kNoAllocMaxDevices];
+static std::once_flag g_noalloc_once[kNoAllocMaxDevices];
+static cudaError_t g_noalloc_err[kNoAllocMaxDevices];
+
+// Host code sees g_noalloc_scratch only as a host-side stand-in; the device
+// address comes from cudaGetSymbolAddress, once per device, with that device
+// current.
+static sla_status noalloc_scratch(int device, void **out) {
+    if (device < 0 || device >= kNoAllocMaxDevices) {
+        set_error("sla_cg_solve_noalloc: device %d beyond the supported %d", device, kNoAllocMaxDevices);
+        return SLA_ERR_UNSUPPORTED;
+    }
+    std::call_once(g_noalloc_once[device], [device] {
+        g_noalloc_err[device] = cudaGetSymbolAddress(&g_noalloc_ptr[device], g_noalloc_scratch);
+    });
+    if (g_noalloc_err[device] != cudaSuccess || g_noalloc_ptr[device] == nullptr) {
+        set_error("sla_cg_solve_noalloc: cudaGetSymbolAddress failed: %s",
+                  cudaGetErrorString(g_noalloc_err[device]));
+        return SLA_ERR_CUDA;
+    }
+    *out = g_noalloc_ptr[device];
+    return SLA_OK;
+}
+
+template <typename T>
+static sla_status noalloc_launch(const Csr &h, const T *vals, const T *b, T *x,
+                                 const sla_cg_opts *o, sla_cg_info info, void *scratch,
+                                 size_t need, cudaStream_t s) {
+    Carver c(scratch);
+    int32_t *diagpos = c.take<int32_t>((size_t)h.n_rows);
+    CgArgs<T> a{};
+    a.n = h.n_rows;
+    a.B = h.batch;
+    a.nnz = h.nnz;
+    a.rowptr = h.rowptr;
+    a.colind = h.colind;
+    a.diagpos = diagpos;
+    a.vals = vals;
+    a.b = b;
+    a.x = x;
+    a.sync = c.take<unsigned>(16);
+    a.sysd = c.take<double>(4 * (size_t)a.B);
+    a.state = c.take<int>(a.B);
+    a.part = c.take<double>(4 * (size_t)a.B * h.ntiles);
+    const size_t vn = (size_t)a.B * a.n;
+    a.r = c.take<T>(vn);
+    a.p = c.take<T>(vn);
+    a.q = c.take<T>(vn);
+    a.d = c.take<T>(vn);
+    if (c.off > need) {
+        set_error("sla_cg_solve_noalloc: internal scratch layout mismatch");
+        return SLA_ERR_CUDA;
+    }
+    a.out_iters = info.iters;
+    a.out_relres = info.relres;
+    a.out_status = info.status;
+    a.rtol = o->rtol;
+    a.atol = o->atol;
+    a.fixed = o->fixed_iters > 0;
+    a.limit = a.fixed ? o->fixed_iters
+                      : (o->max_iter > 0 ? o->max_iter : (a.n < 10000 ? 10 * a.n : 100000));
+    a.precond = o->precond ? 1 : 0;
+    a.x0_given = o->x0_given ? 1 : 0;
+    a.timeout_ns = o->wait_timeout_ns > 0 ? o->wait_timeout_ns : kDefaultTimeoutNs;
+    a.tile_rows = h.tile_rows;
+    a.ntiles = h.ntiles;
+    // the previous call's arrival counter and flags must not leak into this one
+    SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
+    sla_status st = diag_positions(h.n_rows, h.rowptr, h.colind, diagpos, s);
+    if (st != SLA_OK) return st;
+    void *args[] = {&a};
+    SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(pick_fn(true, h.dtype, h.lanes), dim3(h.grid_blocks),
+                                               dim3(kCgThreads), args, 0, s));
+    return SLA_OK;
+}
+
+}  // namespace sla
+
+extern "C" sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t *rowptr,
+                                           const int32_t *colind, int32_t batch, sla_dtype dtype,
+                                           const void *vals, const void *b, void *x,
+                                           const sla_cg_opts *opts, sla_cg_info info,
+                                           void *stream) {
+    clear_error();
+    SLA_REQUIRE(n >= 0 && nnz >= 0 && nnz <= 0x7fffffff, "sla_cg_solve_noalloc: bad sizes n=%d nnz=%lld",
+                n, (long long)nnz);
+    SLA_REQUIRE(batch >= 1, "sla_cg_solve_noalloc: batch must be >= 1");
+    SLA_REQUIRE(dtype == SLA_F64 || dtype == SLA_F32, "sla_cg_solve_noalloc: bad dtype %d", (int)dtype);
+    sla_status st = check_opts(opts);
+    if (st != SLA_OK) return st;
+    SLA_REQUIRE(opts->strategy != SLA_STRATEGY_BLOCK,
+                "sla_cg_solve_noalloc: runs the grid solver only");
+    cudaStream_t s = as_stream(stream);
+    if (n == 0) {
+        info_fill_kernel<<<(batch + 255) / 256, 256, 0, s>>>(batch, info.iters, info.relres, info.status);
+        SLA_CHECK_LAUNCH();
+        return SLA_OK;
+    }
+    SLA_REQUIRE(rowptr && (nnz == 0 || colind) && vals && b && x, "sla_cg_solve_noalloc: NULL pointer");
+    // A handle description on the host stack: no device memory is involved.
+    Csr h;
+    h.n_rows = h.n_cols = n;
+    h.nnz = nnz;
+    h.batch = batch;
+    h.dtype = dtype;
+    h.rowptr = rowptr;
+    h.colind = colind;
+    h.lanes = lanes_for_mean((double)nnz / n);
+    SLA_CHECK_CUDA(cudaGetDevice(&h.device));
+    SLA_CHECK_CUDA(cudaDeviceGetAttribute(&h.num_sms, cudaDevAttrMultiProcessorCount, h.device));
+    int per_sm = 0;
+    SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, pick_fn(true, dtype, h.lanes), kCgThreads, 0));
+    per_sm = per_sm < 2 ? per_sm : 2;
+    if (per_sm < 1) {
+        set_error("sla_cg_solve_noalloc: persistent kernel cannot be resident");
+        return SLA_ERR_CUDA;
+    }
+    h.grid_blocks = per_sm * h.num_sms;
+    layout(&h, h.grid_blocks, &h.tile_rows, &h.ntiles);
+    const int ntot = batch * h.ntiles;
+    if ((ntot + h.grid_blocks - 1) / h.grid_blocks > kMaxLocalTiles) {
+        set_error("sla_cg_solve_noalloc: batch of %d systems too large for one launch", batch);
+        return SLA_ERR_UNSUPPORTED;
+    }
+    const size_t ts = dtype_size(dtype), B = batch, rows = (size_t)n;
+    const size_t need = align_up(rows * 4) + align_up(64) + align_up(4 * B * 8) + align_up(B * 4) +
+                        align_up(4 * (size_t)ntot * 8) + 4 * align_up(B * rows * ts);
+    SLA_REQUIRE(need <= kNoAllocScratchBytes,
+                "sla_cg_solve_noalloc: %d system(s) of %d rows need %zu bytes of scratch; the "
+                "built-in limit is %zu bytes (use sla_cg_solve with a caller workspace)",
+                batch, n, need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    st = noalloc_scratch(h.device, &scratch);
+    if (st != SLA_OK) return st;
+    if (dtype == SLA_F64)
+        return noalloc_launch<double>(h, (const double *)vals, (const double *)b, (double *)x, opts,
+                                      info, scratch, need, s);
+    return noalloc_launch<float>(h, (const float *)vals, (const float *)b, (float *)x, opts, info,
+                                 scratch, need, s);
 }

@@ -258,6 +258,37 @@ sla_status sla_csr_check(int32_t n_rows, int32_t n_cols, int64_t nnz,
                          const int32_t *rowptr, const int32_t *colind,
                          int32_t need_diag, int64_t *result, void *stream);
 
+/*
+ * Allocation-free variant of sla_cg_solve.  The pages have no counterpart: it
+ * exists for callers that may not allocate device memory while they solve
+ * (runtimes that reserve all device memory up front and hand it out
+ * themselves, loops that cannot afford the device-wide synchronisation that
+ * cudaMalloc/cudaFree may imply, plugins that must not call their host's
+ * allocator).  It needs no handle and no workspace: it runs the persistent
+ * grid solver with vectors in global memory, and its scratch (synchronisation
+ * words, partial sums, diagonal positions, the r, p, q, M^-1 vectors) lives in
+ * one static device array of 16 MiB that every GPU loading this library keeps
+ * until the process exits.
+ *   - The first call on a device performs a one-time set-up (it looks up the
+ *     array's device address with that device current); make that first call
+ *     before any stream capture.
+ *   - Sizes whose scratch exceeds 16 MiB (about 4 + 4*sizeof(T) bytes per row
+ *     and system, plus 32 bytes per tile) are rejected with SLA_ERR_INVALID
+ *     and a message giving both sizes; it never allocates, not even then.
+ *   - Every call on a device shares the array, which keeps what the last call
+ *     left: the call clears what must start at zero, and calls whose kernels
+ *     overlap on the GPU (other streams, other host threads) race on it.
+ *   - The pattern is not validated (see sla_csr_check); rowptr/colind must be
+ *     a valid square CSR pattern.
+ * Arguments and outcomes are those of sla_cg_solve (rowptr[n+1], colind[nnz],
+ * vals [B][nnz], b and x [B][n], all device; opts->strategy must not be
+ * SLA_STRATEGY_BLOCK).
+ */
+sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t *rowptr,
+                                const int32_t *colind, int32_t batch, sla_dtype dtype,
+                                const void *vals, const void *b, void *x,
+                                const sla_cg_opts *opts, sla_cg_info info, void *stream);
+
 /* Message for the last non-OK status on this host thread ("" if none). */
 const char *sla_last_error_string(void);
 
