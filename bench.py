@@ -129,15 +129,39 @@ class ClockSampler:
 
 _WORKLOAD = {}
 
+WORKLOADS = ("c2", "c1", "c3", "c4", "c5", "c5rcm")
+CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12}
 
-def oracle_sample(dtype_name: str, k_iters: int):
-    """Oracle on a bounded sample of the step: k forward + k adjoint iterations + gradient."""
+
+def load_workload(name: str, rank: int = 0):
+    """The synthetic workload `name`; every rank gets its own seed (replicas)."""
+    from differentiable_sparse_linear_csr_b200 import workloads as W
+    key = (name, rank)
+    if key not in _WORKLOAD:
+        if name == "c1":
+            w = W.c1_poisson64(seed=1 + 10 * rank)
+        elif name == "c2":
+            w = W.c2_poisson1024(seed=2 + 10 * rank, N=N_GRID, iters=ITERS)
+        elif name == "c3":
+            w = W.c3_diffusion3d(seed=3 + 10 * rank)
+        elif name == "c4":
+            w = W.c4_batched(seed=4 + 10 * rank)
+        elif name == "c5":
+            w = W.c5_knn(seed=5 + 10 * rank)
+        elif name == "c5rcm":
+            w = W.c5_knn(seed=5 + 10 * rank, order="rcm")
+        else:
+            raise ValueError(name)
+        _WORKLOAD[key] = w
+    return _WORKLOAD[key]
+
+
+def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2"):
+    """Oracle on a bounded sample of the step: k forward + k adjoint iterations +
+    gradient, on system 0 of the workload."""
     import numpy as np
     from oracle import oracle as O
-    from differentiable_sparse_linear_csr_b200 import workloads as W
-    if "c2" not in _WORKLOAD:
-        _WORKLOAD["c2"] = W.c2_poisson1024(N=N_GRID, iters=ITERS)
-    w = _WORKLOAD["c2"]
+    w = load_workload(name)
     npdt = np.float64 if dtype_name == "f64" else np.float32
     v, b, xs = w.values[0].astype(npdt), w.b[0].astype(npdt), w.xstar[0].astype(npdt)
     O.build()
@@ -155,10 +179,10 @@ def run_reference(args):
         return 0
     k = args.ref_iters
     for _ in range(args.warmup):
-        oracle_sample(args.dtype, k)
+        oracle_sample(args.dtype, k, args.workload)
     total_it, total_t = 0, 0.0
     for _ in range(args.steps):
-        _, dt = oracle_sample(args.dtype, k)
+        _, dt = oracle_sample(args.dtype, k, args.workload)
         total_it += 2 * k
         total_t += dt
     v = total_it / total_t
@@ -169,19 +193,22 @@ def run_reference(args):
             "config": workload_config(args),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"each step: {k} forward + {k} adjoint PCG iterations + "
-                                       "value gradient of the 1024x1024 Poisson system"},
+                                       f"value gradient of system 0 of workload {args.workload}"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def workload_config(args):
-    n = N_GRID * N_GRID
-    return {"workload": f"2-D 5-point Dirichlet Poisson {N_GRID}x{N_GRID}: fixed {ITERS} forward + "
-                        f"{ITERS} adjoint Jacobi-PCG iterations + sparse value gradient",
-            "n": n, "nnz": 5 * n - 4 * N_GRID, "batch": 1, "value_dtype": args.dtype,
-            "l2": "flushed between steps (write of a 256 MiB buffer)",
-            "parallelism": f"replicas x{int(os.environ.get('WORLD_SIZE', '1'))}"}
+def workload_config(args, w=None):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if w is None:
+        w = load_workload(args.workload)
+    mode = (f"fixed {w.fixed_iters} forward + {w.fixed_iters} adjoint" if w.fixed_iters
+            else f"forward and adjoint to relative residual {w.rtol:g}")
+    return {"workload": f"{w.description}: {mode} Jacobi-PCG iterations + sparse value gradient",
+            "name": args.workload, "n": int(w.n), "nnz": int(w.nnz), "batch": int(w.batch),
+            "value_dtype": args.dtype, "l2": "flushed between steps (write of a 256 MiB buffer)",
+            "parallelism": f"replicas x{world}"}
 
 
 def main():
@@ -192,12 +219,13 @@ def main():
     ap.add_argument("--impl", default="sla", choices=["sla", "reference"])
     ap.add_argument("--dtype", default="f64", choices=["f64", "f32"])
     ap.add_argument("--ref-iters", type=int, default=40)
-    ap.add_argument("--cpu-iters", type=int, default=300)
+    ap.add_argument("--cpu-iters", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--strategy", type=int, default=0)
-    ap.add_argument("--iters", type=int, default=ITERS,
-                    help="iterations per solve; only for short profiler captures")
+    ap.add_argument("--iters", type=int, default=0,
+                    help="override the fixed iteration count (short profiler captures)")
+    ap.add_argument("--workload", default="c2", choices=WORKLOADS)
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -221,33 +249,33 @@ def main():
 
     dt = torch.float64 if args.dtype == "f64" else torch.float32
     vbytes = 8 if args.dtype == "f64" else 4
-    w = W.c2_poisson1024(seed=2 + rank, N=N_GRID, iters=ITERS)
-    n, nnz = w.n, w.nnz
+    w = load_workload(args.workload, rank)
+    n, nnz, B = w.n, w.nnz, w.batch
+    fixed = args.iters if args.iters > 0 else w.fixed_iters
     A = sla.CSR(torch.from_numpy(w.rowptr).to(dev), torch.from_numpy(w.colind).to(dev),
-                dtype=dt, symmetric=True)
+                batch=B, dtype=dt, symmetric=True)
     vals = torch.from_numpy(w.values).to(dev, dt).contiguous()
     b = torch.from_numpy(w.b).to(dev, dt).contiguous()
     xs = torch.from_numpy(w.xstar).to(dev, dt).contiguous()
-    x = torch.empty(1, n, dtype=dt, device=dev)
-    g = torch.empty(1, n, dtype=dt, device=dev)
-    lam = torch.empty(1, n, dtype=dt, device=dev)
-    G = torch.empty(1, nnz, dtype=dt, device=dev)
-    info = [torch.empty(1, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
-    cinfo = L.make_info(*info)
+    x = torch.empty(B, n, dtype=dt, device=dev)
+    g = torch.empty(B, n, dtype=dt, device=dev)
+    lam = torch.empty(B, n, dtype=dt, device=dev)
+    G = torch.empty(B, nnz, dtype=dt, device=dev)
+    finfo = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    ainfo = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
     ws = torch.empty(L.sla_workspace_bytes(A.handle, L.SLA_OP_ADJOINT), dtype=torch.uint8, device=dev)
-    iters = args.iters
-    opts = L.make_opts(fixed_iters=iters, strategy=args.strategy)
+    opts = L.make_opts(rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
     def step(e=None):
         if e: e[0].record(stream)
-        L.sla_cg_solve(A.handle, vals, b, x, opts, cinfo, ws)
+        L.sla_cg_solve(A.handle, vals, b, x, opts, L.make_info(*finfo), ws)
         if e: e[1].record(stream)
         torch.sub(x, xs, out=g)                       # dL/dx of L = 0.5 ||x - x*||^2
         if e: e[2].record(stream)
-        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, cinfo, ws)
+        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, L.make_info(*ainfo), ws)
         if e: e[3].record(stream)
         L.sla_grad_values(A.handle, lam, x, G, 0)
         if e: e[4].record(stream)
@@ -273,11 +301,17 @@ def main():
     fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
     adj_ms = [e[2].elapsed_time(e[3]) for e in events]
     grad_ms = [e[3].elapsed_time(e[4]) for e in events]
+    # every step does the same work (deterministic solver): iterations of the last one
+    fwd_it = int(finfo[0].sum().item())
+    adj_it = int(ainfo[0].sum().item())
+    statuses = sorted(set(finfo[2].tolist()) | set(ainfo[2].tolist()))
+    per_step = torch.tensor([float(fwd_it + adj_it)], dtype=torch.float64, device=dev)
     total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+        dist.all_reduce(per_step, op=dist.ReduceOp.SUM)
     total_ms = float(total_ms.item())
-    iters_done = 2 * iters * args.steps * world
+    iters_done = float(per_step.item()) * args.steps
     value = iters_done / (total_ms / 1000.0)
 
     # ---- end to end through the public API, host buffers, loss read back
@@ -295,7 +329,7 @@ def main():
             bd.copy_(bh, non_blocking=True)
             xd.copy_(xh, non_blocking=True)
             vv = vd.requires_grad_(True)
-            xx = A.solve(vv, bd, fixed_iters=iters, strategy=args.strategy)
+            xx = A.solve(vv, bd, rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
             loss = 0.5 * ((xx - xd) ** 2).sum()
             loss.backward()
             vv.grad = None
@@ -328,30 +362,37 @@ def main():
     if rank == 0:
         peak, peak_kind = measured_hbm_peak()
         it_bytes = per_iteration_bytes(n, nnz, vbytes)
-        cg_launch_ms = statistics.mean(fwd_ms + adj_ms)
-        achieved = iters * it_bytes / (cg_launch_ms / 1000.0) / 1e9
-        traffic = profile_traffic(f"cg_grid_kernel_c2_{args.dtype}")
+        cg_ms = statistics.mean(fwd_ms) + statistics.mean(adj_ms)
+        achieved = (fwd_it + adj_it) * it_bytes / (cg_ms / 1000.0) / 1e9
+        props = A.props
+        variant = ("block-per-system, vectors in shared memory" if (args.strategy == 2 or
+                   (args.strategy == 0 and props.block_fits)) else
+                   "persistent grid, x, r, M^-1 on chip" if props.grid_onchip else
+                   "persistent grid, vectors in HBM")
+        traffic = profile_traffic(f"cg_kernel_{args.workload}_{args.dtype}")
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                "kernel": "cg_grid_kernel (persistent PCG, one launch per solve, %s)"
-                          % ("x, r, M^-1 on chip" if A.props.grid_onchip else "vectors in HBM"),
-                "algorithmic_bytes_per_launch": iters * it_bytes,
-                "launch_ms": cg_launch_ms}
-        gb = grad_bytes(n, nnz, vbytes)
+                "kernel": f"PCG solve kernel ({variant}), one launch per solve",
+                "algorithmic_bytes_per_launch": (fwd_it + adj_it) * it_bytes / 2,
+                "bytes_per_iteration": it_bytes,
+                "launch_ms": cg_ms / 2}
+        gb = grad_bytes(n, nnz, vbytes) * B
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            v_cpu, t_cpu = oracle_sample(args.dtype, args.cpu_iters)
+            k = args.cpu_iters if args.cpu_iters > 0 else CPU_ITERS[args.workload]
+            v_cpu, t_cpu = oracle_sample(args.dtype, k, args.workload)
             cpu = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
-                   "sample": f"{args.cpu_iters} forward + {args.cpu_iters} adjoint PCG iterations + "
-                             f"value gradient of the same system, single-threaded C ({t_cpu:.1f} s)"}
+                   "sample": f"{k} forward + {k} adjoint PCG iterations + value gradient of "
+                             f"system 0, single-threaded C ({t_cpu:.1f} s)"}
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-                "config": workload_config(args),
+                "config": workload_config(args, w),
                 "fwd_adj_grad_ms": statistics.mean(step_ms),
                 "forward_ms": statistics.mean(fwd_ms), "adjoint_ms": statistics.mean(adj_ms),
                 "grad_ms": statistics.mean(grad_ms),
+                "forward_iters": fwd_it, "adjoint_iters": adj_it, "statuses": statuses,
                 "grad_gbs": gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 3 * args.steps,

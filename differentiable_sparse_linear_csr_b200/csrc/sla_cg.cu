@@ -53,6 +53,9 @@ struct CgArgs {
     int limit, fixed, precond, x0_given;
     long long timeout_ns;
     int tile_rows, ntiles;
+    const int32_t *sell_ptr, *sell_cols;   // sliced layout of the pattern (SELL kernels)
+    const T *sell_vals;                     // [B][sell_nnz] values in that layout
+    int64_t sell_nnz;
 };
 
 // ------------------------------------------------------------ helpers ----
@@ -166,7 +169,7 @@ __device__ void give_up(const CgArgs<T> &a) {
 // them itself from the shared partials; ONCHIP keeps x, r and M^-1 of its one
 // tile in shared memory and q in registers (RPT rows a thread), so only A and
 // p travel through L2/HBM each iteration.
-template <typename T, int LANES, bool ONCHIP, int RPT, int NT>
+template <typename T, int LANES, bool ONCHIP, int RPT, int NT, bool SELL>
 __global__ void __launch_bounds__(NT, ONCHIP ? 1 : 2)
 cg_grid_kernel(CgArgs<T> a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -302,7 +305,18 @@ cg_grid_kernel(CgArgs<T> a) {
             const T *vs = a.vals + (int64_t)s * a.nnz;
             const T *pg = a.p + (int64_t)s * n;
             double acc[1] = {0.0};
-            if constexpr (ONCHIP) {
+            if constexpr (ONCHIP && SELL) {
+                const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
+#pragma unroll
+                for (int j = 0; j < RPT; ++j) {
+                    const int i = r0 + tid + j * NT;
+                    if (i < r1) {
+                        const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i);
+                        qreg[j] = qi;
+                        acc[0] += (double)pg[i] * (double)qi;
+                    }
+                }
+            } else if constexpr (ONCHIP) {
 #pragma unroll
                 for (int j = 0; j < RPT; ++j) {
                     const int i = r0 + tid + j * NT;
@@ -311,6 +325,14 @@ cg_grid_kernel(CgArgs<T> a) {
                         qreg[j] = qi;
                         acc[0] += (double)pg[i] * (double)qi;
                     }
+                }
+            } else if constexpr (SELL) {
+                const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
+                T *qg = a.q + (int64_t)s * n;
+                for (int i = r0 + tid; i < r1; i += NT) {
+                    const T qi = sell_row<true>(a.sell_ptr, a.sell_cols, svals, pg, i);
+                    qg[i] = qi;
+                    acc[0] += (double)pg[i] * (double)qi;
                 }
             } else {
                 T *qg = a.q + (int64_t)s * n;
@@ -580,11 +602,15 @@ constexpr int kOnchipThreads = 1024;
 
 template <typename T, int L>
 static const void *grid_fn() {
-    return reinterpret_cast<const void *>(&cg_grid_kernel<T, L, false, 1, kCgThreads>);
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, L, false, 1, kCgThreads, false>);
 }
-template <typename T, int RPT>
+template <typename T>
+static const void *grid_sell_fn() {
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, false, 1, kCgThreads, true>);
+}
+template <typename T, int RPT, bool SELL>
 static const void *onchip_fn() {
-    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads>);
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads, SELL>);
 }
 template <typename T, int L>
 static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L>); }
@@ -600,15 +626,20 @@ static const void *pick_fn(bool grid, sla_dtype dt, int lanes) {
     return f;
 }
 
-static const void *pick_onchip(sla_dtype dt, int rpt) {
+static const void *pick_onchip(sla_dtype dt, int rpt, bool sell) {
     if (dt == SLA_F64) {
-        if (rpt <= 4) return onchip_fn<double, 4>();
-        if (rpt <= 8) return onchip_fn<double, 8>();
-        return onchip_fn<double, 16>();
+        if (rpt <= 4) return sell ? onchip_fn<double, 4, true>() : onchip_fn<double, 4, false>();
+        return sell ? onchip_fn<double, 8, true>() : onchip_fn<double, 8, false>();
     }
-    if (rpt <= 4) return onchip_fn<float, 4>();
-    if (rpt <= 8) return onchip_fn<float, 8>();
-    return onchip_fn<float, 16>();
+    if (rpt <= 4) return sell ? onchip_fn<float, 4, true>() : onchip_fn<float, 4, false>();
+    if (rpt <= 8) return sell ? onchip_fn<float, 8, true>() : onchip_fn<float, 8, false>();
+    return sell ? onchip_fn<float, 16, true>() : onchip_fn<float, 16, false>();
+}
+
+static const void *pick_grid(const Csr *h, bool sell) {
+    if (h->onchip) return pick_onchip(h->dtype, h->onchip_rpt, sell);
+    if (sell) return h->dtype == SLA_F64 ? grid_sell_fn<double>() : grid_sell_fn<float>();
+    return pick_fn(true, h->dtype, h->lanes);
 }
 
 // Tile layout: tiles never straddle systems, and B * ntiles <= blocks whenever
@@ -647,9 +678,11 @@ sla_status cg_configure(Csr *h) {
         const size_t smem = 3 * (size_t)tr * ts;
         const int rpt_cap = h->dtype == SLA_F64 ? 8 : 16;   // beyond this the q registers spill
         if ((int64_t)h->batch * nt <= h->num_sms && rpt <= rpt_cap && smem + 16384 <= (size_t)optin) {
-            const void *f = pick_onchip(h->dtype, rpt);
-            SLA_CHECK_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                optin - 16384));
+            for (int sv = 0; sv < 2; ++sv)
+                SLA_CHECK_CUDA(cudaFuncSetAttribute(pick_onchip(h->dtype, rpt, sv != 0),
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    optin - 16384));
+            const void *f = pick_onchip(h->dtype, rpt, true);
             int per_sm = 0;
             SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kOnchipThreads, smem));
             if (per_sm >= 1) {
@@ -688,6 +721,7 @@ static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
     const size_t B = h->batch, n = h->n_rows, ntot = B * (size_t)h->ntiles;
     size_t b = align_up(64) + align_up(4 * B * 8) + align_up(B * 4) + align_up(4 * ntot * 8);
     b += 4 * align_up(B * n * ts);
+    if (h->has_sell) b += align_up(B * (size_t)h->sell_nnz * ts);
     if (adjoint && !(h->flags & SLA_FLAG_SYMMETRIC)) b += align_up(B * (size_t)h->nnz * ts);
     return b;
 }
@@ -695,7 +729,8 @@ static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
 template <typename T>
 static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind,
                             const int32_t *diagpos, const T *vals, const T *b, T *x,
-                            const sla_cg_opts *o, sla_cg_info info, Carver &c, cudaStream_t s) {
+                            const sla_cg_opts *o, sla_cg_info info, Carver &c, cudaStream_t s,
+                            bool pattern_is_forward) {
     CgArgs<T> a{};
     a.n = h->n_rows;
     a.B = h->batch;
@@ -743,10 +778,20 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
                       "use smaller batches", a.B, a.n, nlt, kMaxLocalTiles);
             return SLA_ERR_UNSUPPORTED;
         }
+        // short rows on the forward pattern: the sliced layout, values laid out now
+        const bool sell = h->has_sell && pattern_is_forward;
+        if (sell) {
+            T *sv = c.take<T>((size_t)a.B * h->sell_nnz);
+            sla_status st = sell_values(h, vals, sv, s);
+            if (st != SLA_OK) return st;
+            a.sell_ptr = h->sell_ptr;
+            a.sell_cols = h->sell_cols;
+            a.sell_vals = sv;
+            a.sell_nnz = h->sell_nnz;
+        }
         SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
         void *args[] = {&a};
-        const void *f = h->onchip ? pick_onchip(h->dtype, h->onchip_rpt)
-                                  : pick_fn(true, h->dtype, h->lanes);
+        const void *f = pick_grid(h, sell);
         SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(f, dim3(h->grid_blocks), dim3(h->grid_threads),
                                                    args, h->grid_smem, s));
     } else {
@@ -803,11 +848,12 @@ static sla_status cg_entry(Csr *h, const void *vals, const void *rhs, void *x,
         if (st != SLA_OK) return st;
         v = vt;
     }
+    const bool forward_pattern = rp == h->rowptr;
     if (h->dtype == SLA_F64)
         return launch_cg<double>(h, rp, ci, dp, (const double *)v, (const double *)rhs,
-                                 (double *)x, o, info, c, s);
+                                 (double *)x, o, info, c, s, forward_pattern);
     return launch_cg<float>(h, rp, ci, dp, (const float *)v, (const float *)rhs, (float *)x, o,
-                            info, c, s);
+                            info, c, s, forward_pattern);
 }
 
 }  // namespace sla

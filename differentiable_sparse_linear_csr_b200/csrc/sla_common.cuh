@@ -97,6 +97,14 @@ struct Csr {
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
+    // Sliced layout of the pattern for the solver's short-row SpMV (see sla_sell.cu):
+    // slices of kSellRows consecutive rows, entry k of the slice's rows stored
+    // together (padded to the slice's longest row).
+    bool has_sell = false;
+    int64_t sell_nnz = 0;              // stored entries including padding
+    int32_t *sell_ptr = nullptr;       // owned [n_slices + 1]: first entry of each slice
+    int32_t *sell_cols = nullptr;      // owned [sell_nnz]: column (own row for padding)
+    int32_t *sell_map = nullptr;       // owned [sell_nnz]: CSR position, -1 for padding
 };
 
 inline size_t dtype_size(sla_dtype dt) { return dt == SLA_F64 ? 8 : 4; }
@@ -117,6 +125,16 @@ sla_status transpose_pattern(int32_t n_rows, int32_t n_cols, int64_t nnz,
 
 // valsT[b][s] = vals[b][permT[s]] for every system (needs the handle's A^T).
 sla_status transpose_values(const Csr *h, const void *vals, void *valsT, cudaStream_t s);
+
+// Device exclusive scan of unsigned counts (n entries; ws >= scan_ws_bytes(n)).
+size_t scan_ws_bytes(int64_t n);
+sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws, cudaStream_t s);
+
+// Sliced layout (built at handle creation for short-row square patterns).
+constexpr int kSellRows = 8;
+sla_status build_sell(Csr *h, cudaStream_t s);
+// vals_sell[b][slot] = vals[b][sell_map[slot]] (0 for padding), every system.
+sla_status sell_values(const Csr *h, const void *vals, void *vals_sell, cudaStream_t s);
 
 // Diagonal positions of a square pattern (kernel; enqueue only).
 sla_status diag_positions(int32_t n, const int32_t *rowptr, const int32_t *colind,

@@ -3,6 +3,7 @@
 // of the torch-sla summary page (technical summary, "Methodology" 1: one
 // matrix, or a batch of value sets sharing one pattern).
 #include <climits>
+#include <cstdlib>
 #include <cstring>
 
 #include "sla_common.cuh"
@@ -268,6 +269,11 @@ extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz
     if (n_rows == n_cols) {
         st = cg_configure(h);
         if (st != SLA_OK) return fail(st);
+        const char *sv = getenv("SLA_SELL");
+        if (h->lanes == 1 && n_rows > 0 && !(sv && sv[0] == '0')) {
+            st = build_sell(h, s);
+            if (st != SLA_OK) return fail(st);
+        }
     }
     if ((flags & SLA_FLAG_BUILD_TRANSPOSE) && !(flags & SLA_FLAG_SYMMETRIC)) {
         st = ensure_transpose(h, s);
@@ -285,6 +291,9 @@ extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     cudaFree(h->colindT);
     cudaFree(h->permT);
     cudaFree(h->diagposT);
+    cudaFree(h->sell_ptr);
+    cudaFree(h->sell_cols);
+    cudaFree(h->sell_map);
     delete h;
     return SLA_OK;
 }

@@ -4,6 +4,8 @@
 // with plain loads because the persistent solver rewrites it between phases.
 #pragma once
 
+#include <type_traits>
+
 #include "sla_common.cuh"
 
 namespace sla {
@@ -53,6 +55,56 @@ __device__ __forceinline__ T row_dot_perm(const int32_t *__restrict__ rowptr,
         const unsigned m = subwarp_mask<LANES>();
 #pragma unroll
         for (int o = LANES / 2; o > 0; o >>= 1) s += __shfl_xor_sync(m, s, o, LANES);
+    }
+    return s;
+}
+
+// Row i of the sliced layout (see sla_sell.cu) times v, one thread per row:
+// entries in stored order, then the slice's zero padding (which adds nothing).
+// R rows i0, i0 + stride, ... are interleaved so that their loads overlap;
+// rows >= row_end are skipped.
+// Loads of the sliced layout's entries.  With STREAM the load bypasses L1
+// (ld.global.nc.L1::no_allocate): in the solver whose vectors live in HBM the
+// matrix streams through once per iteration and L1 is better left to the
+// gathered vector; where the matrix stays in L2 the default allocating load is
+// faster (a slice step uses half a 128-byte line, the next step the other half).
+template <bool STREAM, typename T>
+__device__ __forceinline__ T sell_load(const T *p) {
+    if constexpr (STREAM) {
+        if constexpr (sizeof(T) == 8) {
+            double v;
+            asm volatile("ld.global.nc.L1::no_allocate.f64 %0, [%1];" : "=d"(v) : "l"(p));
+            return (T)v;
+        } else if constexpr (std::is_same<T, float>::value) {
+            float v;
+            asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+            return v;
+        } else {
+            int v;
+            asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
+            return (T)v;
+        }
+    } else {
+        return __ldg(p);
+    }
+}
+
+// Row i of the sliced layout (see sla_sell.cu) times v, one thread per row:
+// the row's entries in stored order, then the slice's zero padding (which adds
+// nothing), so the sum equals row_dot<T, 1>.  One row at a time per thread:
+// interleaving a thread's rows spreads its gathers of v and measured slower.
+template <bool STREAM, typename T>
+__device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
+                                      const int32_t *__restrict__ cols,
+                                      const T *__restrict__ vals, const T *v, int i) {
+    const int sl = i / kSellRows;
+    const int b0 = __ldg(sptr + sl);
+    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
+    const int base = b0 + i % kSellRows;
+    T s = T(0);
+    for (int k = 0; k < w; ++k) {
+        const int t = base + k * kSellRows;
+        s += sell_load<STREAM>(vals + t) * v[sell_load<STREAM>(cols + t)];
     }
     return s;
 }

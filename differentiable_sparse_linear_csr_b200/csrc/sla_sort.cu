@@ -59,7 +59,7 @@ __global__ void scan_add_kernel(unsigned *out, const unsigned *offs, int64_t n) 
     if (i < n) out[i] += offs[i / kScanTile];
 }
 
-static size_t scan_ws_bytes(int64_t n) {
+size_t scan_ws_bytes(int64_t n) {
     size_t b = 256;
     while (n > kScanTile) {
         n = (n + kScanTile - 1) / kScanTile;
@@ -68,7 +68,7 @@ static size_t scan_ws_bytes(int64_t n) {
     return b + 2 * 256;
 }
 
-static sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws,
+sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws,
                                  cudaStream_t s) {
     if (n <= 0) return SLA_OK;
     const int64_t nb = (n + kScanTile - 1) / kScanTile;

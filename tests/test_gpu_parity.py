@@ -251,12 +251,19 @@ def _cases():
     yield "c4x24", w.rowptr, w.colind, w.values, w.b
 
 
-@pytest.mark.parametrize("strategy,onchip", [(L.SLA_STRATEGY_GRID, "1"), (L.SLA_STRATEGY_GRID, "0"),
-                                              (L.SLA_STRATEGY_BLOCK, "1")])
+SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
+    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "0", "1"),
+    (L.SLA_STRATEGY_GRID, "1", "0"), (L.SLA_STRATEGY_GRID, "0", "0"),
+    (L.SLA_STRATEGY_BLOCK, "1", "1")]
+
+
+@pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
 @pytest.mark.parametrize("dtype", [torch.float64, torch.float32])
-def test_pcg_fixed_iterations_parity(strategy, onchip, dtype, monkeypatch):
-    """Both grid variants (x, r, M^-1 on chip or in HBM) and the block solver."""
+def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch):
+    """Every grid variant (x, r, M^-1 on chip or in HBM; sliced or CSR rows) and
+    the block solver."""
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    monkeypatch.setenv("SLA_SELL", sell)
     npdt = np.float64 if dtype == torch.float64 else np.float32
     tol = TOL_X64 if dtype == torch.float64 else TOL_X32
     for name, rp, ci, v, b in _cases():
@@ -274,11 +281,11 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, dtype, monkeypatch):
             assert max(rel_rows(H(x), xo)) < tol, (name, k)
 
 
-@pytest.mark.parametrize("strategy,onchip", [(L.SLA_STRATEGY_GRID, "1"), (L.SLA_STRATEGY_GRID, "0"),
-                                              (L.SLA_STRATEGY_BLOCK, "1")])
-def test_pcg_tolerance_mode_parity(strategy, onchip, monkeypatch):
+@pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
+def test_pcg_tolerance_mode_parity(strategy, onchip, sell, monkeypatch):
     """Iteration counts agree within max(2, 1%); iterates agree at the oracle's count."""
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    monkeypatch.setenv("SLA_SELL", sell)
     for name, rp, ci, v, b in _cases():
         B = v.shape[0]
         A = make(rp, ci, B=B)
