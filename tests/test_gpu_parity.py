@@ -251,10 +251,17 @@ def _cases():
     yield "c4x24", w.rowptr, w.colind, w.values, w.b
 
 
-SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
+SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced layout[+bulk-copy stages])
     (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "0", "1"),
+    (L.SLA_STRATEGY_GRID, "0", "1-nostage"),
     (L.SLA_STRATEGY_GRID, "1", "0"), (L.SLA_STRATEGY_GRID, "0", "0"),
     (L.SLA_STRATEGY_BLOCK, "1", "1")]
+
+
+def _variant_env(monkeypatch, onchip, sell):
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    monkeypatch.setenv("SLA_SELL", sell[0])
+    monkeypatch.setenv("SLA_STAGE", "0" if sell.endswith("nostage") else "1")
 
 
 @pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
@@ -262,8 +269,7 @@ SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
 def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch):
     """Every grid variant (x, r, M^-1 on chip or in HBM; sliced or CSR rows) and
     the block solver."""
-    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
-    monkeypatch.setenv("SLA_SELL", sell)
+    _variant_env(monkeypatch, onchip, sell)
     npdt = np.float64 if dtype == torch.float64 else np.float32
     tol = TOL_X64 if dtype == torch.float64 else TOL_X32
     for name, rp, ci, v, b in _cases():
@@ -284,8 +290,7 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
 @pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
 def test_pcg_tolerance_mode_parity(strategy, onchip, sell, monkeypatch):
     """Iteration counts agree within max(2, 1%); iterates agree at the oracle's count."""
-    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
-    monkeypatch.setenv("SLA_SELL", sell)
+    _variant_env(monkeypatch, onchip, sell)
     for name, rp, ci, v, b in _cases():
         B = v.shape[0]
         A = make(rp, ci, B=B)
