@@ -173,6 +173,22 @@ def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2"):
     return 2 * k_iters / dt, dt
 
 
+def reduce_over_ranks(total_ms: float, iters_per_step: float, device):
+    """Across ranks: the slowest rank's time (max) and every rank's work (sum).
+
+    Replicas solve independent systems, so the job's throughput is all ranks'
+    iterations over the slowest rank's time.  Single-rank runs pass through.
+    """
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    w = torch.tensor([float(iters_per_step)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(w.item())
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -305,13 +321,8 @@ def main():
     fwd_it = int(finfo[0].sum().item())
     adj_it = int(ainfo[0].sum().item())
     statuses = sorted(set(finfo[2].tolist()) | set(ainfo[2].tolist()))
-    per_step = torch.tensor([float(fwd_it + adj_it)], dtype=torch.float64, device=dev)
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-        dist.all_reduce(per_step, op=dist.ReduceOp.SUM)
-    total_ms = float(total_ms.item())
-    iters_done = float(per_step.item()) * args.steps
+    total_ms, per_step = reduce_over_ranks(sum(step_ms), fwd_it + adj_it, dev)
+    iters_done = per_step * args.steps
     value = iters_done / (total_ms / 1000.0)
 
     # ---- end to end through the public API, host buffers, loss read back
@@ -351,10 +362,8 @@ def main():
             e1.record(stream)
             torch.cuda.synchronize()
             e2e_ms += e0.elapsed_time(e1)
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = {"value": iters_done / (float(t.item()) / 1000.0), "unit": UNIT,
+        e2e_total, _ = reduce_over_ranks(e2e_ms, 0.0, dev)
+        e2e = {"value": iters_done / (e2e_total / 1000.0), "unit": UNIT,
                "h2d_bytes_per_step": int(vh.numel() * vh.element_size() + bh.numel() * bh.element_size()
                                          + xh.numel() * xh.element_size()),
                "d2h_bytes_per_step": 8}

@@ -251,17 +251,15 @@ def _cases():
     yield "c4x24", w.rowptr, w.colind, w.values, w.b
 
 
-SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced layout[+bulk-copy stages])
+SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
     (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "0", "1"),
-    (L.SLA_STRATEGY_GRID, "0", "1-nostage"),
     (L.SLA_STRATEGY_GRID, "1", "0"), (L.SLA_STRATEGY_GRID, "0", "0"),
     (L.SLA_STRATEGY_BLOCK, "1", "1")]
 
 
 def _variant_env(monkeypatch, onchip, sell):
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
-    monkeypatch.setenv("SLA_SELL", sell[0])
-    monkeypatch.setenv("SLA_STAGE", "0" if sell.endswith("nostage") else "1")
+    monkeypatch.setenv("SLA_SELL", sell)
 
 
 @pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
