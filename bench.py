@@ -374,6 +374,9 @@ def main():
         cg_ms = statistics.mean(fwd_ms) + statistics.mean(adj_ms)
         achieved = (fwd_it + adj_it) * it_bytes / (cg_ms / 1000.0) / 1e9
         props = A.props
+        uses_grid = not (args.strategy == 2 or (args.strategy == 0 and props.block_fits))
+        # per solve: the solver kernel (+ the sliced-value gather); then the gradient
+        launches_per_step = 2 * (1 + (1 if (uses_grid and props.sliced) else 0)) + 1
         variant = ("block-per-system, vectors in shared memory" if (args.strategy == 2 or
                    (args.strategy == 0 and props.block_fits)) else
                    "persistent grid, x, r, M^-1 on chip" if props.grid_onchip else
@@ -404,7 +407,7 @@ def main():
                 "forward_iters": fwd_it, "adjoint_iters": adj_it, "statuses": statuses,
                 "grad_gbs": gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 3 * args.steps,
+                "gpu_launches": launches_per_step * args.steps,
                 "clocks": clock_info}
         print(json.dumps(line), flush=True)
     if world > 1:

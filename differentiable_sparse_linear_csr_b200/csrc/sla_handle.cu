@@ -316,6 +316,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->has_transpose = h->has_transpose ? 1 : 0;
     p->grid_onchip = h->onchip ? 1 : 0;
     p->grid_tile_rows = h->tile_rows;
+    p->sliced = h->has_sell ? 1 : 0;
     return SLA_OK;
 }
 

@@ -126,6 +126,8 @@ typedef struct {
                                  the environment variable SLA_GRID_ONCHIP=0, read at
                                  creation, turns this variant off */
     int32_t grid_tile_rows;   /* rows of one grid-solver tile */
+    int32_t sliced;           /* 1 if the grid solver uses the 8-row sliced layout (one
+                                 extra value-gather kernel per solve) */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */
