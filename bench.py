@@ -377,7 +377,8 @@ def main():
         uses_grid = not (args.strategy == 2 or (args.strategy == 0 and props.block_fits))
         # per solve: the solver kernel (+ the sliced-value gather); then the gradient
         launches_per_step = 2 * (1 + (1 if (uses_grid and props.sliced) else 0)) + 1
-        variant = ("block-per-system, vectors in shared memory" if (args.strategy == 2 or
+        variant = (("block-per-system, whole system in shared memory" if props.block_resident else
+                    "block-per-system, vectors in shared memory") if (args.strategy == 2 or
                    (args.strategy == 0 and props.block_fits)) else
                    "persistent grid, x, r, M^-1 on chip" if props.grid_onchip else
                    "persistent grid, vectors in HBM")

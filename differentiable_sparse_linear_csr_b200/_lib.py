@@ -51,7 +51,8 @@ class sla_csr_props(ctypes.Structure):
                 ("row_mean", ctypes.c_double), ("lanes", ctypes.c_int32),
                 ("grid_blocks", ctypes.c_int32), ("block_fits", ctypes.c_int32),
                 ("has_transpose", ctypes.c_int32), ("grid_onchip", ctypes.c_int32),
-                ("grid_tile_rows", ctypes.c_int32), ("sliced", ctypes.c_int32)]
+                ("grid_tile_rows", ctypes.c_int32), ("sliced", ctypes.c_int32),
+                ("block_resident", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p

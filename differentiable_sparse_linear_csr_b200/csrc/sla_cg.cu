@@ -24,7 +24,10 @@
 //    shared memory (small systems, large batches): no device-wide barrier.
 #include <cmath>
 #include <cstdlib>
+#include <algorithm>
+#include <climits>
 #include <mutex>
+#include <vector>
 
 #include "sla_rows.cuh"
 
@@ -53,6 +56,8 @@ struct CgArgs {
     int limit, fixed, precond, x0_given;
     long long timeout_ns;
     int tile_rows, ntiles;
+    const int32_t *dep_lo, *dep_hi;        // tiles whose p a tile gathers (null: use a barrier)
+    unsigned *pflag;                        // [ntiles] iteration whose p a tile has written
     const int32_t *sell_ptr, *sell_cols;   // sliced layout of the pattern (SELL kernels)
     const T *sell_vals;                     // [B][sell_nnz] values in that layout
     int64_t sell_nnz;
@@ -151,6 +156,41 @@ __device__ __forceinline__ bool grid_sync(unsigned *sync, unsigned &target, long
     return *flag != 0;
 }
 
+__device__ __forceinline__ void st_release_u32(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until tiles lo..hi (at most 32) have published p of iteration k: warp 0
+// polls them in parallel with acquire loads, bounded like grid_sync.  Every
+// thread of the block must call it; false means leave the kernel.
+__device__ __forceinline__ bool wait_tiles(const unsigned *pflag, int lo, int hi, unsigned k,
+                                           unsigned *sync, long long timeout_ns, int *flag) {
+    if (threadIdx.x < 32) {
+        const int t = lo + (int)threadIdx.x;
+        int ok = 1;
+        const unsigned long long t0 = global_timer_ns();
+        unsigned spins = 0;
+        while (true) {
+            const bool ready = t > hi || ld_acquire_u32(pflag + t) >= k;
+            if (__all_sync(0xffffffffu, ready)) break;
+            if ((spins++ & 7u) == 0) {
+                int bad = 0;
+                if (threadIdx.x == 0)
+                    bad = ld_acquire_u32(sync + 2) != 0 ||
+                          (long long)(global_timer_ns() - t0) > timeout_ns;
+                if (__shfl_sync(0xffffffffu, bad, 0)) {
+                    if (threadIdx.x == 0) atomicExch(sync + 2, 1u);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        if (threadIdx.x == 0) *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
 template <typename T>
 __device__ void give_up(const CgArgs<T> &a) {
     // A wait ran out: every system this block owns reports it.
@@ -187,6 +227,9 @@ cg_grid_kernel(CgArgs<T> a) {
     // With one system spread over every block, each block sees every decision;
     // otherwise the count of active systems decides when the loop ends.
     const bool local_end = (a.B == 1 && a.ntiles >= G);
+    // p-ready flags replace the barrier after the direction update when each
+    // tile's gathers reach only a few tiles (one system spread over all blocks).
+    const bool tile_flags = local_end && a.dep_lo != nullptr;
     double *P0 = a.part, *P1 = P0 + ntot, *P2 = P1 + ntot, *P3 = P2 + ntot;
     const int n = a.n;
     unsigned target = 0;
@@ -301,6 +344,12 @@ cg_grid_kernel(CgArgs<T> a) {
             if (l_state[lt] != kActive) continue;
             const int tile = blockIdx.x + lt * G;
             const int s = tile / a.ntiles, tt = tile % a.ntiles;
+            if (tile_flags && k > 0 &&
+                !wait_tiles(a.pflag, __ldg(a.dep_lo + tt), __ldg(a.dep_hi + tt), (unsigned)k,
+                            a.sync, a.timeout_ns, &flag)) {
+                give_up(a);
+                return;
+            }
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
             const T *vs = a.vals + (int64_t)s * a.nnz;
             const T *pg = a.p + (int64_t)s * n;
@@ -448,6 +497,10 @@ cg_grid_kernel(CgArgs<T> a) {
             }
             __syncthreads();
             if (tid == 0) {
+                if (tile_flags && go_on) {
+                    __threadfence();
+                    st_release_u32(a.pflag + tt, (unsigned)k);
+                }
                 if (go_on) {
                     l_rho[lt] = rho_new;
                     l_rr[lt] = rr;
@@ -457,7 +510,10 @@ cg_grid_kernel(CgArgs<T> a) {
                 }
             }
         }
-        if (local_end) {
+        if (tile_flags) {
+            __syncthreads();
+            more = l_state[0] == kActive;
+        } else if (local_end) {
             if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
             more = l_state[0] == kActive;
         } else {
@@ -477,7 +533,10 @@ cg_grid_kernel(CgArgs<T> a) {
 }
 
 // ------------------------------------------------------ block kernel ----
-template <typename T, int LANES>
+// One block per system (a block loops over systems).  With MRES the whole
+// system lives in shared memory: the shared pattern is loaded once per block,
+// a system's values once per solve, and the iterations touch no global memory.
+template <typename T, int LANES, bool MRES>
 __global__ void __launch_bounds__(kCgThreads)
 cg_block_kernel(CgArgs<T> a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -487,17 +546,33 @@ cg_block_kernel(CgArgs<T> a) {
     const int n = a.n;
     T *xs = reinterpret_cast<T *>(smem_raw);
     T *rs = xs + n, *ps = rs + n, *qs = ps + n, *ds = qs + n;
+    // matrix-resident layout: values, then column indices, then row pointers
+    T *vals_s = ds + n;
+    int32_t *cols_s = reinterpret_cast<int32_t *>(vals_s + (MRES ? a.nnz : 0));
+    int32_t *rp_s = cols_s + (MRES ? a.nnz : 0);
+    if constexpr (MRES) {
+        for (int64_t t = tid; t < a.nnz; t += kCgThreads) cols_s[t] = __ldg(a.colind + t);
+        for (int i = tid; i <= n; i += kCgThreads) rp_s[i] = __ldg(a.rowptr + i);
+    }
 
     for (int s = blockIdx.x; s < a.B; s += gridDim.x) {
         const T *vs = a.vals + (int64_t)s * a.nnz;
         const T *bs = a.b + (int64_t)s * n;
         T *xg = a.x + (int64_t)s * n;
         __syncthreads();
+        if constexpr (MRES) {
+            for (int64_t t = tid; t < a.nnz; t += kCgThreads) vals_s[t] = __ldg(vs + t);
+            __syncthreads();
+        }
+        auto spmv_row = [&](const T *v, int i) -> T {
+            if constexpr (MRES) return row_dot_shared<T, LANES>(rp_s, cols_s, vals_s, v, i, lane);
+            else return row_dot<T, LANES>(a.rowptr, a.colind, vs, v, i, lane);
+        };
         if (a.x0_given) {
             for (int i = tid; i < n; i += kCgThreads) xs[i] = xg[i];
             __syncthreads();
             for (int i = sub; i < n; i += NSUB) {
-                const T v = row_dot<T, LANES>(a.rowptr, a.colind, vs, xs, i, lane);
+                const T v = spmv_row(xs, i);
                 if (lane == 0) qs[i] = v;
             }
             __syncthreads();
@@ -544,7 +619,7 @@ cg_block_kernel(CgArgs<T> a) {
         while (st == kActive) {
             double sg = 0.0;
             for (int i = sub; i < n; i += NSUB) {
-                const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, ps, i, lane);
+                const T qi = spmv_row(ps, i);
                 if (lane == 0) {
                     qs[i] = qi;
                     sg += (double)ps[i] * (double)qi;
@@ -612,8 +687,19 @@ template <typename T, int RPT, bool SELL>
 static const void *onchip_fn() {
     return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads, SELL>);
 }
-template <typename T, int L>
-static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L>); }
+template <typename T, int L, bool MRES = false>
+static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L, MRES>); }
+
+static const void *pick_block(sla_dtype dt, int lanes, bool mres) {
+    const void *f = nullptr;
+    with_lanes(lanes, [&](auto L) -> sla_status {
+        constexpr int LN = decltype(L)::value;
+        if (dt == SLA_F64) f = mres ? block_fn<double, LN, true>() : block_fn<double, LN, false>();
+        else f = mres ? block_fn<float, LN, true>() : block_fn<float, LN, false>();
+        return SLA_OK;
+    });
+    return f;
+}
 
 static const void *pick_fn(bool grid, sla_dtype dt, int lanes) {
     const void *f = nullptr;
@@ -661,11 +747,30 @@ sla_status cg_configure(Csr *h) {
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
     h->block_smem = 5 * (size_t)n * ts;
     h->block_fits = n > 0 && h->block_smem + 2048 <= (size_t)optin;
+    h->block_mres = false;
+    h->block_grid = 4 * h->num_sms;
     if (h->block_fits) {
         // the same ceiling for every handle, so one handle never lowers another's
         SLA_CHECK_CUDA(cudaFuncSetAttribute(pick_fn(false, h->dtype, h->lanes),
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             optin - 2048));
+        // the whole system (values, pattern, vectors) in shared memory when it fits
+        const size_t mres = h->block_smem + (size_t)h->nnz * (ts + 4) + ((size_t)n + 1) * 4;
+        const char *e = getenv("SLA_BLOCK_RESIDENT");
+        if (mres + 2048 <= (size_t)optin && !(e && e[0] == '0')) {
+            const void *f = pick_block(h->dtype, h->lanes, true);
+            SLA_CHECK_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                optin - 2048));
+            int per_sm = 0;
+            SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kCgThreads, mres));
+            // Only when the whole batch runs in one resident wave: with more systems
+            // than resident blocks, more concurrent (non-resident) blocks win.
+            if (per_sm >= 1 && h->batch <= per_sm * h->num_sms) {
+                h->block_mres = true;
+                h->block_smem = mres;
+                h->block_grid = per_sm * h->num_sms;   // each block keeps its pattern copy
+            }
+        }
     }
     // On-chip variant: one 1024-thread block per SM, x, r, M^-1 of the block's
     // rows in shared memory, at most 16 rows a thread.
@@ -716,14 +821,75 @@ sla_status cg_configure(Csr *h) {
     return SLA_OK;
 }
 
+// Range of tiles whose rows a tile's columns reach (one system): per tile the
+// smallest and largest column index over its entries, divided by tile_rows.
+__global__ void tile_deps_kernel(int n, int tile_rows, const int32_t *__restrict__ rowptr,
+                                 const int32_t *__restrict__ colind, int32_t *lo, int32_t *hi) {
+    __shared__ int smin[32], smax[32];
+    const int tt = blockIdx.x;
+    const int r0 = tt * tile_rows, r1 = min(n, r0 + tile_rows);
+    int cmin = INT_MAX, cmax = -1;
+    for (int t = rowptr[r0] + threadIdx.x; t < rowptr[r1]; t += blockDim.x) {
+        const int c = colind[t];
+        cmin = min(cmin, c);
+        cmax = max(cmax, c);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+        cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    }
+    if ((threadIdx.x & 31) == 0) { smin[threadIdx.x >> 5] = cmin; smax[threadIdx.x >> 5] = cmax; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { cmin = min(cmin, smin[w]); cmax = max(cmax, smax[w]); }
+        cmin = min(cmin, smin[0]);
+        cmax = max(cmax, smax[0]);
+        // a tile always depends on itself (its own p enters p.q)
+        lo[tt] = cmax < 0 ? tt : min(tt, cmin / tile_rows);
+        hi[tt] = cmax < 0 ? tt : max(tt, cmax / tile_rows);
+    }
+}
+
+// Dependency ranges for p-ready flags (single-system handles whose tiles each
+// reach at most 32 tiles); otherwise the solver keeps its third barrier.
+sla_status cg_tile_deps(Csr *h, cudaStream_t s) {
+    if (h->batch != 1 || h->n_rows == 0 || h->ntiles < h->grid_blocks) return SLA_OK;
+    const char *e = getenv("SLA_TILE_FLAGS");
+    if (e && e[0] == '0') return SLA_OK;
+    SLA_CHECK_CUDA(cudaMalloc(&h->dep_lo, (size_t)h->ntiles * sizeof(int32_t)));
+    SLA_CHECK_CUDA(cudaMalloc(&h->dep_hi, (size_t)h->ntiles * sizeof(int32_t)));
+    tile_deps_kernel<<<h->ntiles, 256, 0, s>>>(h->n_rows, h->tile_rows, h->rowptr, h->colind,
+                                                h->dep_lo, h->dep_hi);
+    SLA_CHECK_LAUNCH();
+    std::vector<int32_t> lo(h->ntiles), hi(h->ntiles);
+    SLA_CHECK_CUDA(cudaMemcpyAsync(lo.data(), h->dep_lo, lo.size() * 4, cudaMemcpyDeviceToHost, s));
+    SLA_CHECK_CUDA(cudaMemcpyAsync(hi.data(), h->dep_hi, hi.size() * 4, cudaMemcpyDeviceToHost, s));
+    SLA_CHECK_CUDA(cudaStreamSynchronize(s));
+    int span = 0;
+    for (int t = 0; t < h->ntiles; ++t) span = std::max(span, hi[t] - lo[t] + 1);
+    if (span > 32) {
+        cudaFree(h->dep_lo);
+        cudaFree(h->dep_hi);
+        h->dep_lo = h->dep_hi = nullptr;
+    }
+    return SLA_OK;
+}
+
 static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
     const size_t ts = dtype_size(h->dtype);
     const size_t B = h->batch, n = h->n_rows, ntot = B * (size_t)h->ntiles;
     size_t b = align_up(64) + align_up(4 * B * 8) + align_up(B * 4) + align_up(4 * ntot * 8);
     b += 4 * align_up(B * n * ts);
     if (h->has_sell) b += align_up(B * (size_t)h->sell_nnz * ts);
+    b += align_up((size_t)h->ntiles * 4);   // p-ready flags
     if (adjoint && !(h->flags & SLA_FLAG_SYMMETRIC)) b += align_up(B * (size_t)h->nnz * ts);
     return b;
+}
+
+// Tile dependencies hold for the pattern they were built from (the forward
+// pattern; the adjoint reuses it only on symmetric handles).
+static bool pattern_is_forward_or_sym(const Csr *h, const int32_t *rowptr) {
+    return rowptr == h->rowptr;
 }
 
 template <typename T>
@@ -763,6 +929,11 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
     a.timeout_ns = o->wait_timeout_ns > 0 ? o->wait_timeout_ns : kDefaultTimeoutNs;
     a.tile_rows = h->tile_rows;
     a.ntiles = h->ntiles;
+    if (h->dep_lo != nullptr && pattern_is_forward_or_sym(h, rowptr)) {
+        a.dep_lo = h->dep_lo;
+        a.dep_hi = h->dep_hi;
+        a.pflag = c.take<unsigned>((size_t)h->ntiles);
+    }
     bool use_grid = true;
     if (o->strategy == SLA_STRATEGY_BLOCK) {
         SLA_REQUIRE(h->block_fits, "sla_cg: block strategy needs 5*n*sizeof(T) bytes of shared memory");
@@ -790,15 +961,15 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             a.sell_nnz = h->sell_nnz;
         }
         SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
+        if (a.pflag) SLA_CHECK_CUDA(cudaMemsetAsync(a.pflag, 0, (size_t)h->ntiles * sizeof(unsigned), s));
         void *args[] = {&a};
         const void *f = pick_grid(h, sell);
         SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(f, dim3(h->grid_blocks), dim3(h->grid_threads),
                                                    args, h->grid_smem, s));
     } else {
-        const int per = h->num_sms * 4;
-        const int grid = a.B < per ? a.B : per;
+        const int grid = a.B < h->block_grid ? a.B : h->block_grid;
         void *args[] = {&a};
-        SLA_CHECK_CUDA(cudaLaunchKernel(pick_fn(false, h->dtype, h->lanes), dim3(grid),
+        SLA_CHECK_CUDA(cudaLaunchKernel(pick_block(h->dtype, h->lanes, h->block_mres), dim3(grid),
                                         dim3(kCgThreads), args, h->block_smem, s));
     }
     return SLA_OK;

@@ -97,6 +97,9 @@ struct Csr {
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
+    bool block_mres = false;           // block solver keeps the whole system in shared memory
+    int32_t *dep_lo = nullptr, *dep_hi = nullptr;  // owned [ntiles]: tiles a tile's gathers reach
+    int32_t block_grid = 0;            // blocks of the block solver (each loops over systems)
     // Sliced layout of the pattern for the solver's short-row SpMV (see sla_sell.cu):
     // slices of kSellRows consecutive rows, entry k of the slice's rows stored
     // together (padded to the slice's longest row).
@@ -133,6 +136,7 @@ sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws
 // Sliced layout (built at handle creation for short-row square patterns).
 constexpr int kSellRows = 8;
 sla_status build_sell(Csr *h, cudaStream_t s);
+sla_status cg_tile_deps(Csr *h, cudaStream_t s);   // in sla_cg.cu
 // vals_sell[b][slot] = vals[b][sell_map[slot]] (0 for padding), every system.
 sla_status sell_values(const Csr *h, const void *vals, void *vals_sell, cudaStream_t s);
 

@@ -268,6 +268,7 @@ extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz
     }
     if (n_rows == n_cols) {
         st = cg_configure(h);
+        if (st == SLA_OK) st = cg_tile_deps(h, s);
         if (st != SLA_OK) return fail(st);
         const char *sv = getenv("SLA_SELL");
         if (h->lanes == 1 && n_rows > 0 && !(sv && sv[0] == '0')) {
@@ -294,6 +295,8 @@ extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     cudaFree(h->sell_ptr);
     cudaFree(h->sell_cols);
     cudaFree(h->sell_map);
+    cudaFree(h->dep_lo);
+    cudaFree(h->dep_hi);
     delete h;
     return SLA_OK;
 }
@@ -317,6 +320,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_onchip = h->onchip ? 1 : 0;
     p->grid_tile_rows = h->tile_rows;
     p->sliced = h->has_sell ? 1 : 0;
+    p->block_resident = h->block_mres ? 1 : 0;
     return SLA_OK;
 }
 

@@ -39,6 +39,21 @@ __device__ __forceinline__ T row_dot(const int32_t *__restrict__ rowptr,
     return s;
 }
 
+// Same product with every array in shared memory (plain loads).
+template <typename T, int LANES>
+__device__ __forceinline__ T row_dot_shared(const int32_t *rowptr, const int32_t *colind,
+                                            const T *vals, const T *v, int i, int lane) {
+    const int t0 = rowptr[i], t1 = rowptr[i + 1];
+    T s = T(0);
+    for (int t = t0 + lane; t < t1; t += LANES) s += vals[t] * v[colind[t]];
+    if constexpr (LANES > 1) {
+        const unsigned m = subwarp_mask<LANES>();
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) s += __shfl_xor_sync(m, s, o, LANES);
+    }
+    return s;
+}
+
 // Same with the values reached through a permutation (A^T's entry s is A's
 // entry perm[s]); used by transposed SpMV on non-symmetric handles.
 template <typename T, int LANES>

@@ -128,6 +128,8 @@ typedef struct {
     int32_t grid_tile_rows;   /* rows of one grid-solver tile */
     int32_t sliced;           /* 1 if the grid solver uses the 8-row sliced layout (one
                                  extra value-gather kernel per solve) */
+    int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
+                                 system in shared memory as well as its vectors */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */
