@@ -374,14 +374,21 @@ def main():
         cg_ms = statistics.mean(fwd_ms) + statistics.mean(adj_ms)
         achieved = (fwd_it + adj_it) * it_bytes / (cg_ms / 1000.0) / 1e9
         props = A.props
-        uses_grid = not (args.strategy == 2 or (args.strategy == 0 and props.block_fits))
+        uses_cluster = args.strategy == 3 or (args.strategy == 0 and props.cluster_fits
+                                              and w.batch * 8 <= 148)
+        uses_grid = not uses_cluster and not (args.strategy == 2 or
+                                              (args.strategy == 0 and props.block_fits))
         # per solve: the solver kernel (+ the sliced-value gather); then the gradient
         launches_per_step = 2 * (1 + (1 if (uses_grid and props.sliced) else 0)) + 1
-        variant = (("block-per-system, whole system in shared memory" if props.block_resident else
-                    "block-per-system, vectors in shared memory") if (args.strategy == 2 or
-                   (args.strategy == 0 and props.block_fits)) else
-                   "persistent grid, x, r, M^-1 on chip" if props.grid_onchip else
-                   "persistent grid, vectors in HBM")
+        if uses_cluster:
+            variant = "thread-block cluster per system, DSMEM"
+        elif not uses_grid:
+            variant = ("block-per-system, whole system in shared memory" if props.block_resident
+                       else "block-per-system, vectors in shared memory")
+        elif props.grid_onchip:
+            variant = "persistent grid, x, r, M^-1 on chip"
+        else:
+            variant = "persistent grid, vectors in HBM"
         traffic = profile_traffic(f"cg_kernel_{args.workload}_{args.dtype}")
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,

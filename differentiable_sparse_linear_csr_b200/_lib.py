@@ -18,7 +18,7 @@ SLA_F64, SLA_F32 = 0, 1
 SLA_OK, SLA_ERR_INVALID, SLA_ERR_CUDA, SLA_ERR_OOM, SLA_ERR_TIMEOUT, SLA_ERR_UNSUPPORTED = range(6)
 SLA_CONVERGED, SLA_NOT_CONVERGED, SLA_BREAKDOWN, SLA_NONFINITE, SLA_FIXED_DONE, SLA_TIMED_OUT = range(6)
 SLA_FLAG_VALIDATE, SLA_FLAG_SYMMETRIC, SLA_FLAG_BUILD_TRANSPOSE = 1, 2, 4
-SLA_STRATEGY_AUTO, SLA_STRATEGY_GRID, SLA_STRATEGY_BLOCK = 0, 1, 2
+SLA_STRATEGY_AUTO, SLA_STRATEGY_GRID, SLA_STRATEGY_BLOCK, SLA_STRATEGY_CLUSTER = 0, 1, 2, 3
 SLA_OP_SPMV, SLA_OP_CG, SLA_OP_ADJOINT, SLA_OP_GRAD = 0, 1, 2, 3
 
 STATUS_NAMES = {0: "converged", 1: "not_converged", 2: "breakdown", 3: "nonfinite",
@@ -52,7 +52,7 @@ class sla_csr_props(ctypes.Structure):
                 ("grid_blocks", ctypes.c_int32), ("block_fits", ctypes.c_int32),
                 ("has_transpose", ctypes.c_int32), ("grid_onchip", ctypes.c_int32),
                 ("grid_tile_rows", ctypes.c_int32), ("sliced", ctypes.c_int32),
-                ("block_resident", ctypes.c_int32)]
+                ("block_resident", ctypes.c_int32), ("cluster_fits", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p

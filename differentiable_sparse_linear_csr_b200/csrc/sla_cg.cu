@@ -24,6 +24,8 @@
 //    shared memory (small systems, large batches): no device-wide barrier.
 #include <cmath>
 #include <cstdlib>
+#include <cooperative_groups.h>
+
 #include <algorithm>
 #include <climits>
 #include <mutex>
@@ -664,6 +666,227 @@ cg_block_kernel(CgArgs<T> a) {
     }
 }
 
+// ---------------------------------------------------- cluster kernel ----
+// One thread-block cluster per system (kClusterCTAs blocks): each block owns a
+// contiguous run of rows and keeps its rows' matrix entries, x, r, M^-1, q and
+// p in its own shared memory for the whole solve.  The SpMV reads other
+// blocks' p through distributed shared memory; cluster-wide sums go through
+// per-block partial slots read over DSMEM in rank order, so every block takes
+// the same decisions.  Waits inside the loop are a software barrier on a
+// counter in rank 0's shared memory, bounded like grid_sync; every exit path
+// ends in one hardware cluster barrier so that no block leaves while another
+// may still read its shared memory.
+constexpr int kClusterCTAs = 8;
+constexpr int kClusterThreads = 512;
+
+__device__ __forceinline__ void red_release_cluster(unsigned *p, unsigned v) {
+    asm volatile("red.release.cluster.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_cluster(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.cluster.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ bool cluster_sync_bounded(unsigned *count0, unsigned *err0, unsigned &target,
+                                                     long long timeout_ns, int *flag) {
+    __syncthreads();
+    target += kClusterCTAs;
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        // the arrive is a release and the poll an acquire at cluster scope; the
+        // block barriers around them order the other threads' shared-memory work
+        red_release_cluster(count0, 1u);
+        const unsigned long long t0 = global_timer_ns();
+        unsigned spins = 0;
+        while ((int)(ld_acquire_cluster(count0) - target) < 0) {
+            if ((spins++ & 7u) == 0) {
+                if (ld_acquire_cluster(err0) != 0) { ok = 0; break; }
+                if ((long long)(global_timer_ns() - t0) > timeout_ns) {
+                    atomicExch(err0, 1u);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        if (ok && ld_acquire_cluster(err0) != 0) ok = 0;
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT)
+cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
+    namespace cgs = cooperative_groups;
+    constexpr int CS = kClusterCTAs;
+    cgs::cluster_group cl = cgs::this_cluster();
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ double red[4 * 33];
+    __shared__ double cpart[2][4];
+    __shared__ unsigned cbar_count, cbar_err;
+    __shared__ int flag;
+    __shared__ double bc[4];
+    __shared__ T *pbase[CS];
+    const int rank = (int)cl.block_rank();
+    const int sys = blockIdx.x / CS;
+    const int tid = threadIdx.x;
+    const int n = a.n;
+    T *p_s = reinterpret_cast<T *>(smem_raw);
+    T *x_s = p_s + rows_cta, *r_s = x_s + rows_cta, *d_s = r_s + rows_cta, *q_s = d_s + rows_cta;
+    T *v_s = q_s + rows_cta;
+    int32_t *c_s = reinterpret_cast<int32_t *>(v_s + nnz_cap);
+    int32_t *rp_s = c_s + nnz_cap;
+
+    if (tid == 0) { cbar_count = 0; cbar_err = 0; }
+    if (tid < CS) pbase[tid] = cl.map_shared_rank(p_s, tid);
+    unsigned *count0 = cl.map_shared_rank(&cbar_count, 0);
+    unsigned *err0 = cl.map_shared_rank(&cbar_err, 0);
+    unsigned target = 0;
+    int exch = 0;
+    cl.sync();   // every block's counters and pointers are set before first use
+
+    const int r0 = rank * rows_cta, r1 = min(n, r0 + rows_cta);
+    const int m = r1 > r0 ? r1 - r0 : 0;
+    const T *vs = a.vals + (int64_t)sys * a.nnz;
+    const T *bs = a.b + (int64_t)sys * n;
+    T *xg = a.x + (int64_t)sys * n;
+    const int t0 = m > 0 ? __ldg(a.rowptr + r0) : 0, t1 = m > 0 ? __ldg(a.rowptr + r1) : 0;
+    for (int i = tid; i <= m; i += NT) rp_s[i] = m > 0 ? __ldg(a.rowptr + r0 + i) - t0 : 0;
+    for (int t = t0 + tid; t < t1; t += NT) {
+        c_s[t - t0] = __ldg(a.colind + t);
+        v_s[t - t0] = __ldg(vs + t);
+    }
+    __syncthreads();
+
+    // cluster-wide sums of NV values: block sums -> this block's slot -> barrier
+    // -> every block adds the CS slots in rank order
+    auto cluster_sums = [&](double *v, int nv) -> bool {
+        double tmp[4] = {v[0], nv > 1 ? v[1] : 0.0, nv > 2 ? v[2] : 0.0, nv > 3 ? v[3] : 0.0};
+        block_sums<NT, 4>(tmp, red);
+        const int slot = exch & 1;
+        if (tid == 0)
+            for (int k = 0; k < 4; ++k) cpart[slot][k] = tmp[k];
+        ++exch;
+        if (!cluster_sync_bounded(count0, err0, target, a.timeout_ns, &flag)) return false;
+        if (tid < 32) {
+            for (int k = 0; k < nv; ++k) {
+                double x = tid < CS ? *cl.map_shared_rank(&cpart[slot][k], tid) : 0.0;
+                x = warp_sum(x);
+                if (tid == 0) bc[k] = x;
+            }
+        }
+        __syncthreads();
+        for (int k = 0; k < nv; ++k) v[k] = bc[k];
+        __syncthreads();
+        return true;
+    };
+    auto gather_p = [&](int j) -> T {
+        const int o = j / rows_cta;
+        return pbase[o][j - o * rows_cta];
+    };
+
+    int st = kActive, k = 0;
+    double relres = 0.0, nb = 0.0, tol = 0.0, rho = 0.0, rr = 0.0;
+    bool alive = true;
+    {   // r = b - A x0 (or b), z = M^-1 r, p = z
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int li = tid; li < m; li += NT) {
+            const int i = r0 + li;
+            const T bi = bs[i];
+            T ri = bi, xi = T(0), dv = T(0);
+            T ax = T(0);
+            for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) {
+                if (c_s[t] == i) dv = v_s[t];
+                if (a.x0_given) ax += v_s[t] * xg[c_s[t]];
+            }
+            if (a.x0_given) {
+                xi = xg[i];
+                ri = bi - ax;
+            }
+            T di = T(1);
+            if (a.precond) {
+                if (!(dv > T(0))) acc[3] += 1.0;
+                di = T(1) / dv;
+            }
+            const T zi = di * ri;
+            x_s[li] = xi;
+            r_s[li] = ri;
+            d_s[li] = di;
+            p_s[li] = zi;
+            acc[0] += (double)bi * (double)bi;
+            acc[1] += (double)ri * (double)zi;
+            acc[2] += (double)ri * (double)ri;
+        }
+        alive = cluster_sums(acc, 4);
+        nb = sqrt(acc[0]);
+        rho = acc[1];
+        rr = acc[2];
+        tol = fmax(a.rtol * nb, a.atol);
+        if (nb == 0.0) st = SLA_CONVERGED;
+        else if (!isfinite(nb)) st = SLA_NONFINITE;
+        else if (a.precond && acc[3] > 0.0) { st = SLA_BREAKDOWN; relres = sqrt(rr) / nb; }
+        else if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; relres = sqrt(rr) / nb; }
+        else if (rr == 0.0) st = SLA_CONVERGED;
+        if (nb == 0.0)
+            for (int li = tid; li < m; li += NT) x_s[li] = T(0);
+    }
+    while (alive && st == kActive) {
+        double sg[1] = {0.0};
+        for (int li = tid; li < m; li += NT) {
+            T qi = T(0);
+            for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) qi += v_s[t] * gather_p(c_s[t]);
+            q_s[li] = qi;
+            sg[0] += (double)p_s[li] * (double)qi;
+        }
+        if (!(alive = cluster_sums(sg, 1))) break;
+        const double sigma = sg[0];
+        if (!isfinite(sigma) || !(sigma > 0.0)) {
+            st = isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE;
+            relres = sqrt(rr) / nb;
+            break;
+        }
+        const double alpha = rho / sigma;
+        const T al = (T)alpha;
+        ++k;
+        double acc[2] = {0.0, 0.0};
+        for (int li = tid; li < m; li += NT) {
+            const T ri = r_s[li] - al * q_s[li];
+            r_s[li] = ri;
+            const T zi = d_s[li] * ri;
+            acc[0] += (double)ri * (double)zi;
+            acc[1] += (double)ri * (double)ri;
+        }
+        if (!(alive = cluster_sums(acc, 2))) break;
+        const double rho_new = acc[0];
+        rr = acc[1];
+        relres = sqrt(rr) / nb;
+        if (!isfinite(rr)) st = SLA_NONFINITE;
+        else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
+        else if (rr == 0.0) st = SLA_CONVERGED;
+        else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
+        const T bt = (T)(rho_new / rho);
+        const bool go_on = st == kActive;
+        for (int li = tid; li < m; li += NT) {
+            const T pi = p_s[li];
+            x_s[li] = x_s[li] + al * pi;
+            if (go_on) p_s[li] = d_s[li] * r_s[li] + bt * pi;
+        }
+        rho = rho_new;
+        if (go_on && !(alive = cluster_sync_bounded(count0, err0, target, a.timeout_ns, &flag))) break;
+    }
+    if (alive)
+        for (int li = tid; li < m; li += NT) xg[r0 + li] = x_s[li];
+    if (rank == 0 && tid == 0) {
+        const int out = alive ? st : SLA_TIMED_OUT;
+        if (a.out_status) a.out_status[sys] = out;
+        if (a.out_iters) a.out_iters[sys] = k;
+        if (a.out_relres) a.out_relres[sys] = relres;
+    }
+    cl.sync();   // no block leaves while another may still read its shared memory
+}
+
 __global__ void info_fill_kernel(int B, int32_t *iters, double *relres, int32_t *status) {
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= B) return;
@@ -689,6 +912,11 @@ static const void *onchip_fn() {
 }
 template <typename T, int L, bool MRES = false>
 static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L, MRES>); }
+
+template <typename T>
+static const void *cluster_fn() {
+    return reinterpret_cast<const void *>(&cg_cluster_kernel<T, kClusterThreads>);
+}
 
 static const void *pick_block(sla_dtype dt, int lanes, bool mres) {
     const void *f = nullptr;
@@ -726,6 +954,15 @@ static const void *pick_grid(const Csr *h, bool sell) {
     if (h->onchip) return pick_onchip(h->dtype, h->onchip_rpt, sell);
     if (sell) return h->dtype == SLA_F64 ? grid_sell_fn<double>() : grid_sell_fn<float>();
     return pick_fn(true, h->dtype, h->lanes);
+}
+
+// One dynamic shared-memory ceiling per kernel for every handle (static shared
+// memory of these kernels stays below 8 KB), so no handle lowers another's.
+static sla_status smem_ceiling(const void *f, int device) {
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    SLA_CHECK_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 8192));
+    return SLA_OK;
 }
 
 // Tile layout: tiles never straddle systems, and B * ntiles <= blocks whenever
@@ -817,6 +1054,46 @@ sla_status cg_configure(Csr *h) {
         h->grid_threads = kCgThreads;
         h->grid_smem = 0;
         layout(h, h->grid_blocks, &h->tile_rows, &h->ntiles);
+    }
+    // Cluster solver: rows split over kClusterCTAs blocks on 32-row boundaries,
+    // each block's matrix slice, vectors and p in its shared memory.
+    h->cluster_fits = false;
+    const char *ce = getenv("SLA_CLUSTER");
+    if (n > 0 && n <= 65536 && !(ce && ce[0] == '0')) {
+        int64_t rc = ((int64_t)n + kClusterCTAs - 1) / kClusterCTAs;
+        rc = (rc + 31) / 32 * 32;
+        std::vector<int32_t> rp((size_t)n + 1);
+        SLA_CHECK_CUDA(cudaMemcpy(rp.data(), h->rowptr, rp.size() * sizeof(int32_t), cudaMemcpyDeviceToHost));
+        int64_t cap = 0;
+        for (int r = 0; r < kClusterCTAs; ++r) {
+            const int64_t a0 = std::min<int64_t>(n, r * rc), a1 = std::min<int64_t>(n, (r + 1) * rc);
+            cap = std::max<int64_t>(cap, (int64_t)rp[a1] - rp[a0]);
+        }
+        const size_t smem = 5 * (size_t)rc * ts + (size_t)cap * (ts + 4) + ((size_t)rc + 1) * 4;
+        if (smem + 8192 <= (size_t)optin) {
+            const void *f = h->dtype == SLA_F64 ? cluster_fn<double>() : cluster_fn<float>();
+            sla_status st = smem_ceiling(f, h->device);
+            if (st != SLA_OK) return st;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(kClusterCTAs);
+            cfg.blockDim = dim3(kClusterThreads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = kClusterCTAs;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int nclusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&nclusters, f, &cfg) == cudaSuccess && nclusters >= 1) {
+                h->cluster_fits = true;
+                h->cluster_rows = (int32_t)rc;
+                h->cluster_nnz = (int32_t)std::max<int64_t>(cap, 1);
+                h->cluster_smem = smem;
+            }
+            cudaGetLastError();
+        }
     }
     return SLA_OK;
 }
@@ -934,14 +1211,35 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
         a.dep_hi = h->dep_hi;
         a.pflag = c.take<unsigned>((size_t)h->ntiles);
     }
-    bool use_grid = true;
+    bool use_grid = true, use_cluster = false;
     if (o->strategy == SLA_STRATEGY_BLOCK) {
         SLA_REQUIRE(h->block_fits, "sla_cg: block strategy needs 5*n*sizeof(T) bytes of shared memory");
         use_grid = false;
+    } else if (o->strategy == SLA_STRATEGY_CLUSTER) {
+        SLA_REQUIRE(h->cluster_fits, "sla_cg: the system does not fit the cluster solver");
+        use_grid = false;
+        use_cluster = true;
     } else if (o->strategy == SLA_STRATEGY_AUTO) {
-        use_grid = !h->block_fits;
+        // a cluster per system while the batch leaves SMs for all clusters at once
+        use_cluster = h->cluster_fits && (int64_t)a.B * kClusterCTAs <= h->num_sms;
+        use_grid = !use_cluster && !h->block_fits;
     }
-    if (use_grid) {
+    if (use_cluster) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)a.B * kClusterCTAs);
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.dynamicSmemBytes = h->cluster_smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kClusterCTAs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        SLA_CHECK_CUDA(cudaLaunchKernelEx(&cfg, cg_cluster_kernel<T, kClusterThreads>, a,
+                                          (int)h->cluster_rows, (int)h->cluster_nnz));
+    } else if (use_grid) {
         const int ntot = a.B * a.ntiles;
         const int nlt = (ntot + h->grid_blocks - 1) / h->grid_blocks;
         if (nlt > kMaxLocalTiles) {
@@ -980,7 +1278,7 @@ static sla_status check_opts(const sla_cg_opts *o) {
     SLA_REQUIRE(o->rtol >= 0.0 && o->atol >= 0.0 && std::isfinite(o->rtol) && std::isfinite(o->atol),
                 "sla_cg: rtol/atol must be finite and >= 0");
     SLA_REQUIRE(o->fixed_iters >= 0, "sla_cg: fixed_iters < 0");
-    SLA_REQUIRE(o->strategy >= 0 && o->strategy <= 2, "sla_cg: unknown strategy %d", o->strategy);
+    SLA_REQUIRE(o->strategy >= 0 && o->strategy <= 3, "sla_cg: unknown strategy %d", o->strategy);
     SLA_REQUIRE(o->reserved == 0, "sla_cg: reserved field must be 0");
     return SLA_OK;
 }

@@ -98,6 +98,10 @@ struct Csr {
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
     bool block_mres = false;           // block solver keeps the whole system in shared memory
+    bool cluster_fits = false;         // one system fits the cluster solver
+    int32_t cluster_rows = 0;          // rows of one cluster block
+    int32_t cluster_nnz = 0;           // most entries any cluster block holds
+    size_t cluster_smem = 0;           // its dynamic shared memory
     int32_t *dep_lo = nullptr, *dep_hi = nullptr;  // owned [ntiles]: tiles a tile's gathers reach
     int32_t block_grid = 0;            // blocks of the block solver (each loops over systems)
     // Sliced layout of the pattern for the solver's short-row SpMV (see sla_sell.cu):

@@ -321,6 +321,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_tile_rows = h->tile_rows;
     p->sliced = h->has_sell ? 1 : 0;
     p->block_resident = h->block_mres ? 1 : 0;
+    p->cluster_fits = h->cluster_fits ? 1 : 0;
     return SLA_OK;
 }
 

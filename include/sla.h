@@ -85,11 +85,14 @@ enum {
                                       on a non-symmetric handle; built lazily otherwise) */
 };
 
-/* Solver strategies (sla_cg_opts.strategy).  AUTO picks by size: one thread
- * block per system when a system's vectors fit in shared memory, else one
- * persistent cooperative grid with device-wide barriers.  The others force a
- * choice (benchmarks and tests). */
-enum { SLA_STRATEGY_AUTO = 0, SLA_STRATEGY_GRID = 1, SLA_STRATEGY_BLOCK = 2 };
+/* Solver strategies (sla_cg_opts.strategy).  AUTO picks by size: one
+ * thread-block cluster per system (matrix slice and vectors in the blocks'
+ * shared memory, p shared over distributed shared memory) for a few systems
+ * that fit a cluster; one thread block per system when a system's vectors fit
+ * in shared memory; else one persistent cooperative grid with device-wide
+ * barriers.  The others force a choice (benchmarks and tests). */
+enum { SLA_STRATEGY_AUTO = 0, SLA_STRATEGY_GRID = 1, SLA_STRATEGY_BLOCK = 2,
+       SLA_STRATEGY_CLUSTER = 3 };
 
 typedef struct {
     double rtol;              /* relative residual target (tolerance mode) */
@@ -130,6 +133,7 @@ typedef struct {
                                  extra value-gather kernel per solve) */
     int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
                                  system in shared memory as well as its vectors */
+    int32_t cluster_fits;     /* 1 if one system fits the cluster solver */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */

@@ -254,7 +254,7 @@ def _cases():
 SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
     (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "0", "1"),
     (L.SLA_STRATEGY_GRID, "1", "0"), (L.SLA_STRATEGY_GRID, "0", "0"),
-    (L.SLA_STRATEGY_BLOCK, "1", "1")]
+    (L.SLA_STRATEGY_BLOCK, "1", "1"), (L.SLA_STRATEGY_CLUSTER, "1", "1")]
 
 
 def _variant_env(monkeypatch, onchip, sell):
@@ -275,6 +275,8 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
         A = make(rp, ci, B=B, dtype=dtype)
         if strategy == L.SLA_STRATEGY_BLOCK and not A.props.block_fits:
             continue
+        if strategy == L.SLA_STRATEGY_CLUSTER and not A.props.cluster_fits:
+            continue
         if strategy == L.SLA_STRATEGY_GRID and onchip == "0":
             assert A.props.grid_onchip == 0
         for k in (1, 7, 60):
@@ -293,6 +295,8 @@ def test_pcg_tolerance_mode_parity(strategy, onchip, sell, monkeypatch):
         B = v.shape[0]
         A = make(rp, ci, B=B)
         if strategy == L.SLA_STRATEGY_BLOCK and not A.props.block_fits:
+            continue
+        if strategy == L.SLA_STRATEGY_CLUSTER and not A.props.cluster_fits:
             continue
         xo, io = O.pcg(rp, ci, v, b, rtol=1e-10)
         x, info = A.cg(T(v), T(b), rtol=1e-10, strategy=strategy)
@@ -319,7 +323,7 @@ def test_results_are_bitwise_reproducible(onchip, monkeypatch):
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     w = W.c1_poisson64()
     A = make(w.rowptr, w.colind)
-    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK):
+    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK, L.SLA_STRATEGY_CLUSTER):
         x1, i1 = A.cg(T(w.values), T(w.b), rtol=1e-10, strategy=strategy)
         x2, i2 = A.cg(T(w.values), T(w.b), rtol=1e-10, strategy=strategy)
         assert torch.equal(x1, x2) and torch.equal(i1.iters, i2.iters)
@@ -423,7 +427,7 @@ def test_edge_cases_match_oracle_outcomes():
     rp, ci, v = W.random_spd(300, 0.02, 4)
     A = make(rp, ci)
     b = W.uniform(4, 0, 300, -1, 1)
-    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK):
+    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK, L.SLA_STRATEGY_CLUSTER):
         x, info = A.cg(T(v), T(np.zeros(300)), strategy=strategy)
         assert H(info.iters)[0] == 0 and H(info.status)[0] == L.SLA_CONVERGED and not H(x).any()
         xs = np.linalg.solve(W.csr_to_dense(rp, ci, v), b)
@@ -446,7 +450,7 @@ def test_edge_cases_match_oracle_outcomes():
     # indefinite matrix: breakdown; negative diagonal: breakdown before any step
     rpi, cii, vi = W.dense_to_csr(np.array([[1.0, 2.0], [2.0, 1.0]]))
     Ai = make(rpi, cii)
-    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK):
+    for strategy in (L.SLA_STRATEGY_GRID, L.SLA_STRATEGY_BLOCK, L.SLA_STRATEGY_CLUSTER):
         _, info = Ai.cg(T(vi), T(np.array([1.0, -1.0])), rtol=1e-12, strategy=strategy)
         _, io = O.pcg(rpi, cii, vi, np.array([1.0, -1.0]), rtol=1e-12)
         assert H(info.status)[0] == io.status[0] == L.SLA_BREAKDOWN
@@ -478,3 +482,25 @@ def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
     x, info = A.cg(T(v), b, fixed_iters=20, strategy=L.SLA_STRATEGY_GRID)
     xo, _ = O.pcg(rp, ci, v, W.normal(2, 0, 300 * 300), fixed_iters=20)
     assert H(info.status)[0] == L.SLA_FIXED_DONE and rel(H(x)[0], xo) < TOL_X64
+
+
+def test_cluster_bounded_wait_times_out_without_hanging():
+    w = W.c1_poisson64()
+    A = make(w.rowptr, w.colind)
+    assert A.props.cluster_fits
+    _, info = A.cg(T(w.values), T(w.b), fixed_iters=400, strategy=L.SLA_STRATEGY_CLUSTER,
+                   wait_timeout_ns=1)
+    assert H(info.status)[0] == L.SLA_TIMED_OUT
+    x, info = A.cg(T(w.values), T(w.b), fixed_iters=20, strategy=L.SLA_STRATEGY_CLUSTER)
+    xo, _ = O.pcg(w.rowptr, w.colind, w.values[0], w.b[0], fixed_iters=20)
+    assert H(info.status)[0] == L.SLA_FIXED_DONE and rel(H(x)[0], xo) < TOL_X64
+
+
+def test_auto_strategy_picks_cluster_for_a_small_single_system():
+    w = W.c1_poisson64()
+    A = make(w.rowptr, w.colind)
+    x, info = A.cg(T(w.values), T(w.b), rtol=1e-10)
+    xo, io = O.pcg(w.rowptr, w.colind, w.values[0], w.b[0], rtol=1e-10)
+    assert abs(int(H(info.iters)[0]) - int(io.iters[0])) <= 2
+    xk, _ = A.cg(T(w.values), T(w.b), fixed_iters=int(io.iters[0]), strategy=L.SLA_STRATEGY_CLUSTER)
+    assert rel(H(xk)[0], xo) < TOL_X64
