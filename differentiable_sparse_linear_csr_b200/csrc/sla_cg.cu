@@ -716,6 +716,18 @@ __device__ __forceinline__ bool cluster_sync_bounded(unsigned *count0, unsigned 
     return *flag != 0;
 }
 
+// p_k = z_{k-1} + beta p_{k-1} with z = M^-1 r, computed the same way (one
+// rounded product, one fused multiply-add) by the owner and by every gatherer.
+template <typename T>
+__device__ __forceinline__ T direction(T d, T r, T p, T beta) {
+    if constexpr (sizeof(T) == 8) return __fma_rn(beta, p, __dmul_rn(d, r));
+    else return __fmaf_rn(beta, p, __fmul_rn(d, r));
+}
+
+// Two cluster-wide synchronisations per iteration: the SpMV of iteration k
+// forms each gathered p_k(j) from the owner's M^-1, r and p_{k-1} (double
+// buffered) instead of waiting for the owner to write p_k; x and r are updated
+// together once alpha is known.
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT)
 cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
@@ -728,19 +740,25 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
     __shared__ unsigned cbar_count, cbar_err;
     __shared__ int flag;
     __shared__ double bc[4];
-    __shared__ T *pbase[CS];
+    __shared__ T *pb[2][CS], *rb[CS], *db[CS];
     const int rank = (int)cl.block_rank();
     const int sys = blockIdx.x / CS;
     const int tid = threadIdx.x;
     const int n = a.n;
-    T *p_s = reinterpret_cast<T *>(smem_raw);
-    T *x_s = p_s + rows_cta, *r_s = x_s + rows_cta, *d_s = r_s + rows_cta, *q_s = d_s + rows_cta;
+    T *p0_s = reinterpret_cast<T *>(smem_raw);
+    T *p1_s = p0_s + rows_cta, *x_s = p1_s + rows_cta, *r_s = x_s + rows_cta, *d_s = r_s + rows_cta;
+    T *q_s = d_s + rows_cta;
     T *v_s = q_s + rows_cta;
     int32_t *c_s = reinterpret_cast<int32_t *>(v_s + nnz_cap);
     int32_t *rp_s = c_s + nnz_cap;
 
     if (tid == 0) { cbar_count = 0; cbar_err = 0; }
-    if (tid < CS) pbase[tid] = cl.map_shared_rank(p_s, tid);
+    if (tid < CS) {
+        pb[0][tid] = cl.map_shared_rank(p0_s, tid);
+        pb[1][tid] = cl.map_shared_rank(p1_s, tid);
+        rb[tid] = cl.map_shared_rank(r_s, tid);
+        db[tid] = cl.map_shared_rank(d_s, tid);
+    }
     unsigned *count0 = cl.map_shared_rank(&cbar_count, 0);
     unsigned *err0 = cl.map_shared_rank(&cbar_err, 0);
     unsigned target = 0;
@@ -760,7 +778,7 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
     }
     __syncthreads();
 
-    // cluster-wide sums of NV values: block sums -> this block's slot -> barrier
+    // cluster-wide sums of nv values: block sums -> this block's slot -> barrier
     // -> every block adds the CS slots in rank order
     auto cluster_sums = [&](double *v, int nv) -> bool {
         double tmp[4] = {v[0], nv > 1 ? v[1] : 0.0, nv > 2 ? v[2] : 0.0, nv > 3 ? v[3] : 0.0};
@@ -782,15 +800,11 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
         __syncthreads();
         return true;
     };
-    auto gather_p = [&](int j) -> T {
-        const int o = j / rows_cta;
-        return pbase[o][j - o * rows_cta];
-    };
 
     int st = kActive, k = 0;
     double relres = 0.0, nb = 0.0, tol = 0.0, rho = 0.0, rr = 0.0;
     bool alive = true;
-    {   // r = b - A x0 (or b), z = M^-1 r, p = z
+    {   // r = b - A x0 (or b), M^-1; p_0 = 0 so that p_1 = z_0
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
         for (int li = tid; li < m; li += NT) {
             const int i = r0 + li;
@@ -814,7 +828,7 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
             x_s[li] = xi;
             r_s[li] = ri;
             d_s[li] = di;
-            p_s[li] = zi;
+            p0_s[li] = T(0);
             acc[0] += (double)bi * (double)bi;
             acc[1] += (double)ri * (double)zi;
             acc[2] += (double)ri * (double)ri;
@@ -832,13 +846,24 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
         if (nb == 0.0)
             for (int li = tid; li < m; li += NT) x_s[li] = T(0);
     }
+    T bt = T(0);   // beta_{k-1}; 0 before the first step
     while (alive && st == kActive) {
+        // SpMV of iteration k+1 with p_{k+1} = z_k + beta_k p_k formed on the fly
+        const int cur = (k + 1) & 1, prev = k & 1;
+        T *pcur = cur ? p1_s : p0_s;
+        const T *pprev = prev ? p1_s : p0_s;
         double sg[1] = {0.0};
         for (int li = tid; li < m; li += NT) {
             T qi = T(0);
-            for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) qi += v_s[t] * gather_p(c_s[t]);
+            for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) {
+                const int j = c_s[t];
+                const int o = j / rows_cta, lj = j - o * rows_cta;
+                qi += v_s[t] * direction(db[o][lj], rb[o][lj], pb[prev][o][lj], bt);
+            }
             q_s[li] = qi;
-            sg[0] += (double)p_s[li] * (double)qi;
+            const T pi = direction(d_s[li], r_s[li], pprev[li], bt);
+            pcur[li] = pi;
+            sg[0] += (double)pi * (double)qi;
         }
         if (!(alive = cluster_sums(sg, 1))) break;
         const double sigma = sg[0];
@@ -847,11 +872,11 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
             relres = sqrt(rr) / nb;
             break;
         }
-        const double alpha = rho / sigma;
-        const T al = (T)alpha;
+        const T al = (T)(rho / sigma);
         ++k;
         double acc[2] = {0.0, 0.0};
         for (int li = tid; li < m; li += NT) {
+            x_s[li] = x_s[li] + al * pcur[li];
             const T ri = r_s[li] - al * q_s[li];
             r_s[li] = ri;
             const T zi = d_s[li] * ri;
@@ -866,15 +891,8 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
         else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
         else if (rr == 0.0) st = SLA_CONVERGED;
         else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
-        const T bt = (T)(rho_new / rho);
-        const bool go_on = st == kActive;
-        for (int li = tid; li < m; li += NT) {
-            const T pi = p_s[li];
-            x_s[li] = x_s[li] + al * pi;
-            if (go_on) p_s[li] = d_s[li] * r_s[li] + bt * pi;
-        }
+        bt = (T)(rho_new / rho);
         rho = rho_new;
-        if (go_on && !(alive = cluster_sync_bounded(count0, err0, target, a.timeout_ns, &flag))) break;
     }
     if (alive)
         for (int li = tid; li < m; li += NT) xg[r0 + li] = x_s[li];
@@ -1069,7 +1087,7 @@ sla_status cg_configure(Csr *h) {
             const int64_t a0 = std::min<int64_t>(n, r * rc), a1 = std::min<int64_t>(n, (r + 1) * rc);
             cap = std::max<int64_t>(cap, (int64_t)rp[a1] - rp[a0]);
         }
-        const size_t smem = 5 * (size_t)rc * ts + (size_t)cap * (ts + 4) + ((size_t)rc + 1) * 4;
+        const size_t smem = 6 * (size_t)rc * ts + (size_t)cap * (ts + 4) + ((size_t)rc + 1) * 4;
         if (smem + 8192 <= (size_t)optin) {
             const void *f = h->dtype == SLA_F64 ? cluster_fn<double>() : cluster_fn<float>();
             sla_status st = smem_ceiling(f, h->device);
