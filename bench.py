@@ -385,6 +385,8 @@ def main():
         elif not uses_grid:
             variant = ("block-per-system, whole system in shared memory" if props.block_resident
                        else "block-per-system, vectors in shared memory")
+        elif props.grid_onchip == 2:
+            variant = "persistent grid, x, r, M^-1 on chip, two barriers an iteration"
         elif props.grid_onchip:
             variant = "persistent grid, x, r, M^-1 on chip"
         else:

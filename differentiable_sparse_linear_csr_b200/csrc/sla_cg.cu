@@ -534,6 +534,176 @@ cg_grid_kernel(CgArgs<T> a) {
     }
 }
 
+// --------------------------------------------- two-sync grid kernel ----
+// The persistent solver for one system with x, r and M^-1 on chip and the
+// sliced layout, with two device-wide barriers per iteration instead of three:
+// the SpMV of iteration k forms p_k(j) = z_{k-1}(j) + beta p_{k-1}(j) per
+// gathered entry from z = M^-1 r (written by each row's owner when it updates
+// r) and the previous direction (p double buffered), and x and r are updated
+// together once alpha is known.  Workspace vectors: a.r holds z, a.p and a.q
+// the two directions.
+template <typename T, int RPT, int NT>
+__global__ void __launch_bounds__(NT, 1)
+cg_grid2_kernel(CgArgs<T> a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ double red[4 * 33];
+    __shared__ int flag;
+    const int tid = threadIdx.x;
+    const int G = gridDim.x;
+    const int n = a.n;
+    const int tile = blockIdx.x;                 // one tile per block, one system
+    const bool has_tile = tile < a.ntiles;
+    const int r0 = tile * a.tile_rows, r1 = has_tile ? min(n, r0 + a.tile_rows) : r0;
+    double *P0 = a.part, *P1 = P0 + a.ntiles, *P2 = P1 + a.ntiles, *P3 = P2 + a.ntiles;
+    T *xs = reinterpret_cast<T *>(smem_raw);
+    T *rs = xs + a.tile_rows, *ds = rs + a.tile_rows;
+    T *zg = a.r, *pbuf[2] = {a.p, a.q};
+    const T *svals = a.sell_vals;
+    unsigned target = 0;
+    T qreg[RPT];
+
+    // ---- init: r = b - A x0 (or b), M^-1, z_0 = M^-1 r_0, p_0 = 0
+    {
+        const T *bs = a.b;
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        if (a.x0_given && has_tile) {
+#pragma unroll
+            for (int j = 0; j < RPT; ++j) {
+                const int i = r0 + tid + j * NT;
+                if (i < r1) qreg[j] = row_dot<T, 1>(a.rowptr, a.colind, a.vals, a.x, i, 0);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int i = r0 + tid + j * NT;
+            if (i < r1) {
+                const T bi = bs[i];
+                const T xi = a.x0_given ? a.x[i] : T(0);
+                const T ri = a.x0_given ? bi - qreg[j] : bi;
+                T di = T(1);
+                if (a.precond) {
+                    const int dp = __ldg(a.diagpos + i);
+                    const T dv = dp >= 0 ? __ldg(a.vals + dp) : T(0);
+                    if (!(dv > T(0))) acc[3] += 1.0;
+                    di = T(1) / dv;
+                }
+                const T zi = di * ri;
+                xs[i - r0] = xi;
+                rs[i - r0] = ri;
+                ds[i - r0] = di;
+                zg[i] = zi;
+                pbuf[0][i] = T(0);
+                acc[0] += (double)bi * (double)bi;
+                acc[1] += (double)ri * (double)zi;
+                acc[2] += (double)ri * (double)ri;
+            }
+        }
+        block_sums<NT, 4>(acc, red);
+        if (tid == 0 && has_tile) {
+            P0[tile] = acc[0];
+            P1[tile] = acc[1];
+            P2[tile] = acc[2];
+            P3[tile] = acc[3];
+        }
+    }
+    if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
+    double nb, tol, rho, rr;
+    int st = kActive;
+    double relres = 0.0;
+    {
+        const double *const arr[4] = {P0, P1, P2, P3};
+        double sum[4];
+        system_sums<NT, 4>(arr, a.ntiles, sum, red);
+        nb = sqrt(sum[0]);
+        rho = sum[1];
+        rr = sum[2];
+        tol = fmax(a.rtol * nb, a.atol);
+        if (nb == 0.0) st = SLA_CONVERGED;
+        else if (!isfinite(nb)) st = SLA_NONFINITE;
+        else if (a.precond && sum[3] > 0.0) { st = SLA_BREAKDOWN; relres = sqrt(rr) / nb; }
+        else if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; relres = sqrt(rr) / nb; }
+        else if (rr == 0.0) st = SLA_CONVERGED;
+        if (nb == 0.0)
+            for (int i = r0 + tid; i < r1; i += NT) xs[i - r0] = T(0);
+    }
+    int k = 0;
+    T bt = T(0);
+    while (st == kActive) {
+        // ---- SpMV with p_{k+1} = z_k + beta_k p_k, partials of p.q
+        const T *pprev = pbuf[k & 1];
+        T *pcur = pbuf[(k + 1) & 1];
+        double acc[1] = {0.0};
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int i = r0 + tid + j * NT;
+            if (i < r1) {
+                const T qi = sell_row_dir<T>(a.sell_ptr, a.sell_cols, svals, zg, pprev, bt, i);
+                qreg[j] = qi;
+                T pi;
+                if constexpr (sizeof(T) == 8) pi = __fma_rn(bt, pprev[i], __dmul_rn(ds[i - r0], rs[i - r0]));
+                else pi = __fmaf_rn(bt, pprev[i], __fmul_rn(ds[i - r0], rs[i - r0]));
+                pcur[i] = pi;
+                acc[0] += (double)pi * (double)qi;
+            }
+        }
+        block_sums<NT, 1>(acc, red);
+        if (tid == 0 && has_tile) P0[tile] = acc[0];
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
+        double sg[1];
+        {
+            const double *const arr[1] = {P0};
+            system_sums<NT, 1>(arr, a.ntiles, sg, red);
+        }
+        const double sigma = sg[0];
+        if (!isfinite(sigma) || !(sigma > 0.0)) {
+            st = isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE;
+            relres = sqrt(rr) / nb;
+            break;
+        }
+        const T al = (T)(rho / sigma);
+        ++k;
+        // ---- x += alpha p; r -= alpha q; z = M^-1 r; partials of r.z, r.r
+        double acc2[2] = {0.0, 0.0};
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int i = r0 + tid + j * NT;
+            if (i < r1) {
+                xs[i - r0] = xs[i - r0] + al * pcur[i];
+                const T ri = rs[i - r0] - al * qreg[j];
+                rs[i - r0] = ri;
+                T zi;
+                if constexpr (sizeof(T) == 8) zi = __dmul_rn(ds[i - r0], ri);
+                else zi = __fmul_rn(ds[i - r0], ri);
+                zg[i] = zi;
+                acc2[0] += (double)ri * (double)zi;
+                acc2[1] += (double)ri * (double)ri;
+            }
+        }
+        block_sums<NT, 2>(acc2, red);
+        if (tid == 0 && has_tile) {
+            P1[tile] = acc2[0];
+            P2[tile] = acc2[1];
+        }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
+        double sum[2];
+        {
+            const double *const arr[2] = {P1, P2};
+            system_sums<NT, 2>(arr, a.ntiles, sum, red);
+        }
+        const double rho_new = sum[0];
+        rr = sum[1];
+        relres = sqrt(rr) / nb;
+        if (!isfinite(rr)) st = SLA_NONFINITE;
+        else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
+        else if (rr == 0.0) st = SLA_CONVERGED;
+        else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
+        bt = (T)(rho_new / rho);
+        rho = rho_new;
+    }
+    for (int i = r0 + tid; i < r1; i += NT) a.x[i] = xs[i - r0];
+    if (blockIdx.x == 0 && tid == 0) finalize(a, 0, st, k, relres, false);
+}
+
 // ------------------------------------------------------ block kernel ----
 // One block per system (a block loops over systems).  With MRES the whole
 // system lives in shared memory: the shared pattern is loaded once per block,
@@ -928,6 +1098,10 @@ template <typename T, int RPT, bool SELL>
 static const void *onchip_fn() {
     return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads, SELL>);
 }
+template <typename T, int RPT>
+static const void *grid2_fn() {
+    return reinterpret_cast<const void *>(&cg_grid2_kernel<T, RPT, kOnchipThreads>);
+}
 template <typename T, int L, bool MRES = false>
 static const void *block_fn() { return reinterpret_cast<const void *>(&cg_block_kernel<T, L, MRES>); }
 
@@ -966,6 +1140,12 @@ static const void *pick_onchip(sla_dtype dt, int rpt, bool sell) {
     if (rpt <= 4) return sell ? onchip_fn<float, 4, true>() : onchip_fn<float, 4, false>();
     if (rpt <= 8) return sell ? onchip_fn<float, 8, true>() : onchip_fn<float, 8, false>();
     return sell ? onchip_fn<float, 16, true>() : onchip_fn<float, 16, false>();
+}
+
+static const void *pick_grid2(sla_dtype dt, int rpt) {
+    if (dt == SLA_F64) return rpt <= 4 ? grid2_fn<double, 4>() : grid2_fn<double, 8>();
+    if (rpt <= 4) return grid2_fn<float, 4>();
+    return rpt <= 8 ? grid2_fn<float, 8>() : grid2_fn<float, 16>();
 }
 
 static const void *pick_grid(const Csr *h, bool sell) {
@@ -1038,10 +1218,10 @@ sla_status cg_configure(Csr *h) {
         const size_t smem = 3 * (size_t)tr * ts;
         const int rpt_cap = h->dtype == SLA_F64 ? 8 : 16;   // beyond this the q registers spill
         if ((int64_t)h->batch * nt <= h->num_sms && rpt <= rpt_cap && smem + 16384 <= (size_t)optin) {
-            for (int sv = 0; sv < 2; ++sv)
-                SLA_CHECK_CUDA(cudaFuncSetAttribute(pick_onchip(h->dtype, rpt, sv != 0),
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    optin - 16384));
+            for (int sv = 0; sv < 3; ++sv)
+                SLA_CHECK_CUDA(cudaFuncSetAttribute(
+                    sv < 2 ? pick_onchip(h->dtype, rpt, sv != 0) : pick_grid2(h->dtype, rpt),
+                    cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 16384));
             const void *f = pick_onchip(h->dtype, rpt, true);
             int per_sm = 0;
             SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kOnchipThreads, smem));
@@ -1053,6 +1233,20 @@ sla_status cg_configure(Csr *h) {
                 h->grid_blocks = h->num_sms;
                 h->tile_rows = tr;
                 h->ntiles = nt;
+                // One system with one tile a block: the two-barrier solver (it
+                // needs the sliced layout, decided after this).  It gathers two
+                // vectors where the three-barrier one gathers one, so it is
+                // taken only while both gathered tiles stay in L1 beside the
+                // on-chip vectors (measured on a 10^6-row 2-D Poisson system:
+                // +5% in fp32, where they fit; -35% in fp64, where they do not).
+                const char *g2 = getenv("SLA_GRID2");
+                int per_sm2 = 0, smem_sm = 0;
+                SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm2, pick_grid2(h->dtype, rpt), kOnchipThreads, smem));
+                cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, h->device);
+                const bool l1_fits = smem + 2 * (size_t)tr * ts <= (size_t)smem_sm;
+                h->grid2 = h->batch == 1 && nt <= h->num_sms && per_sm2 >= 1 &&
+                           (l1_fits || (g2 && g2[0] == '2')) && !(g2 && g2[0] == '0');
             }
         }
     }
@@ -1279,7 +1473,8 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
         SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
         if (a.pflag) SLA_CHECK_CUDA(cudaMemsetAsync(a.pflag, 0, (size_t)h->ntiles * sizeof(unsigned), s));
         void *args[] = {&a};
-        const void *f = pick_grid(h, sell);
+        const void *f = sell && h->grid2 && a.B == 1 ? pick_grid2(h->dtype, h->onchip_rpt)
+                                                     : pick_grid(h, sell);
         SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(f, dim3(h->grid_blocks), dim3(h->grid_threads),
                                                    args, h->grid_smem, s));
     } else {

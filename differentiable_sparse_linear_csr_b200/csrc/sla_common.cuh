@@ -94,6 +94,7 @@ struct Csr {
     bool block_fits = false;           // one system fits the block-per-system solver
     bool onchip = false;               // grid solver keeps x, r, M^-1 in shared memory
     int32_t onchip_rpt = 0;            // rows a thread in the on-chip grid solver
+    bool grid2 = false;                // single system, on chip, sliced: two barriers an iteration
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block

@@ -317,7 +317,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_blocks = h->grid_blocks;
     p->block_fits = h->block_fits ? 1 : 0;
     p->has_transpose = h->has_transpose ? 1 : 0;
-    p->grid_onchip = h->onchip ? 1 : 0;
+    p->grid_onchip = h->onchip ? (h->grid2 && h->has_sell ? 2 : 1) : 0;
     p->grid_tile_rows = h->tile_rows;
     p->sliced = h->has_sell ? 1 : 0;
     p->block_resident = h->block_mres ? 1 : 0;

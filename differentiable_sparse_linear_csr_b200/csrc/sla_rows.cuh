@@ -124,6 +124,30 @@ __device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
     return s;
 }
 
+// Row of the sliced layout times the direction p_k = z + beta p_prev, formed
+// per gathered entry with one fused multiply-add (the owner of each row forms
+// the same value the same way from its own M^-1 r, rounded once, as z).
+template <typename T>
+__device__ __forceinline__ T sell_row_dir(const int32_t *__restrict__ sptr,
+                                          const int32_t *__restrict__ cols,
+                                          const T *__restrict__ vals, const T *z, const T *pprev,
+                                          T beta, int i) {
+    const int sl = i / kSellRows;
+    const int b0 = __ldg(sptr + sl);
+    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
+    const int base = b0 + i % kSellRows;
+    T s = T(0);
+    for (int k = 0; k < w; ++k) {
+        const int t = base + k * kSellRows;
+        const int c = __ldg(cols + t);
+        T pj;
+        if constexpr (sizeof(T) == 8) pj = __fma_rn(beta, pprev[c], z[c]);
+        else pj = __fmaf_rn(beta, pprev[c], z[c]);
+        s += __ldg(vals + t) * pj;
+    }
+    return s;
+}
+
 // Dispatch a functor templated on LANES.
 template <typename F>
 sla_status with_lanes(int lanes, F &&f) {

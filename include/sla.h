@@ -126,8 +126,10 @@ typedef struct {
     int32_t block_fits;       /* 1 if one system fits the block-per-system solver */
     int32_t has_transpose;    /* 1 once A^T's pattern is built */
     int32_t grid_onchip;      /* 1 if the grid solver keeps x, r, M^-1 on chip (else in HBM);
-                                 the environment variable SLA_GRID_ONCHIP=0, read at
-                                 creation, turns this variant off */
+                                 2 if, besides, a single system on the sliced layout runs
+                                 the two-barrier form (directions formed while gathered);
+                                 the environment variables SLA_GRID_ONCHIP=0 and
+                                 SLA_GRID2=0, read at creation, turn these variants off */
     int32_t grid_tile_rows;   /* rows of one grid-solver tile */
     int32_t sliced;           /* 1 if the grid solver uses the 8-row sliced layout (one
                                  extra value-gather kernel per solve) */

@@ -251,14 +251,18 @@ def _cases():
     yield "c4x24", w.rowptr, w.colind, w.values, w.b
 
 
-SOLVER_VARIANTS = [  # (strategy, on-chip grid vectors, sliced short-row layout)
-    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "0", "1"),
-    (L.SLA_STRATEGY_GRID, "1", "0"), (L.SLA_STRATEGY_GRID, "0", "0"),
-    (L.SLA_STRATEGY_BLOCK, "1", "1"), (L.SLA_STRATEGY_CLUSTER, "1", "1")]
+# (strategy, on-chip grid vectors, sliced short-row layout); on-chip "3" keeps
+# the vectors on chip but turns the two-barrier single-system form off
+SOLVER_VARIANTS = [
+    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"),
+    (L.SLA_STRATEGY_GRID, "0", "1"), (L.SLA_STRATEGY_GRID, "1", "0"),
+    (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_BLOCK, "1", "1"),
+    (L.SLA_STRATEGY_CLUSTER, "1", "1")]
 
 
 def _variant_env(monkeypatch, onchip, sell):
-    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    monkeypatch.setenv("SLA_GRID_ONCHIP", "0" if onchip == "0" else "1")
+    monkeypatch.setenv("SLA_GRID2", "0" if onchip == "3" else "1")
     monkeypatch.setenv("SLA_SELL", sell)
 
 
@@ -279,6 +283,10 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
             continue
         if strategy == L.SLA_STRATEGY_GRID and onchip == "0":
             assert A.props.grid_onchip == 0
+        if strategy == L.SLA_STRATEGY_GRID and onchip == "3":
+            assert A.props.grid_onchip in (0, 1)
+        if strategy == L.SLA_STRATEGY_GRID and onchip == "1" and B == 1 and A.props.sliced:
+            assert A.props.grid_onchip == 2, name
         for k in (1, 7, 60):
             x, info = A.cg(T(v.astype(npdt)), T(b.astype(npdt)), fixed_iters=k, strategy=strategy)
             xo, io = O.pcg(rp, ci, v.astype(npdt), b.astype(npdt), fixed_iters=k)
@@ -470,9 +478,9 @@ def test_single_unknown_and_empty_matrix():
     assert x.shape == (2, 0) and np.all(H(info.status) == 0) and np.all(H(info.iters) == 0)
 
 
-@pytest.mark.parametrize("onchip", ["1", "0"])
+@pytest.mark.parametrize("onchip", ["1", "3", "0"])
 def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
-    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.poisson2d(300)
     A = make(rp, ci)
     b = T(W.normal(2, 0, 300 * 300))
