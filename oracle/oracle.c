@@ -164,6 +164,56 @@ int32_t orc_dense_lu_solve(int32_t n, double *a, double *b)
     return 0;
 }
 
+/*
+ * Pattern positions of an undirected edge list, for the edge-weighted Laplacian
+ * of inverse coefficient learning (torch-sla summary page, "Experimental
+ * results", end-to-end application: spatially varying conductivities of a
+ * Poisson problem recovered through A.solve by gradient descent).  Edge e joins
+ * ei[e] and ej[e]; its two entries (i, j) and (j, i) are found by scanning rows
+ * i and j.  owner[t] = the edge whose weight entry t carries, -1 for entries
+ * that carry none (the diagonal and entries no edge names).  Every failure is
+ * a pair (code, index); the smallest code, then the smallest index, is
+ * returned with *where = that index (0 and -1 when the edges are valid):
+ *   1 an endpoint outside [0, n)           (index: the edge)
+ *   2 a self loop, i == j                  (the edge)
+ *   3 entry (i, j) or (j, i) not stored    (the edge)
+ *   4 an unordered pair an earlier edge already named  (the later edge)
+ *   5 a row without a diagonal entry       (the row)
+ */
+int32_t orc_edge_slots(int32_t n, const int32_t *rowptr, const int32_t *colind,
+                       int64_t n_edges, const int32_t *ei, const int32_t *ej,
+                       int64_t *slot_ij, int64_t *slot_ji, int64_t *owner, int64_t *where)
+{
+    int32_t best = 0;
+    int64_t best_at = -1;
+#define ORC_FAIL(c, at) do { if (best == 0 || (c) < best || ((c) == best && (at) < best_at)) \
+                                 { best = (c); best_at = (at); } } while (0)
+    for (int64_t t = 0; t < (int64_t)rowptr[n]; ++t) owner[t] = -1;
+    for (int64_t e = 0; e < n_edges; ++e) {
+        const int32_t i = ei[e], j = ej[e];
+        slot_ij[e] = slot_ji[e] = -1;
+        if (i < 0 || i >= n || j < 0 || j >= n) { ORC_FAIL(1, e); continue; }
+        if (i == j) { ORC_FAIL(2, e); continue; }
+        for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t)
+            if (colind[t] == j) slot_ij[e] = t;
+        for (int32_t t = rowptr[j]; t < rowptr[j + 1]; ++t)
+            if (colind[t] == i) slot_ji[e] = t;
+        if (slot_ij[e] < 0 || slot_ji[e] < 0) { ORC_FAIL(3, e); continue; }
+        if (owner[slot_ij[e]] >= 0 || owner[slot_ji[e]] >= 0) { ORC_FAIL(4, e); continue; }
+        owner[slot_ij[e]] = e;
+        owner[slot_ji[e]] = e;
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t found = 0;
+        for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t)
+            if (colind[t] == i) found = 1;
+        if (!found) ORC_FAIL(5, i);
+    }
+#undef ORC_FAIL
+    *where = best_at;
+    return best;
+}
+
 #define T double
 #define SUFFIX f64
 #include "oracle_body.h"

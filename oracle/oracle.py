@@ -69,6 +69,12 @@ def _L():
             getattr(_lib, f"orc_grad_values_{sfx}").argtypes = [i32, P, P, P, P, P, i32]
             getattr(_lib, f"orc_coo_to_csr_{sfx}").argtypes = [i32, i32, i64, P, P, P, P, P, P, P]
             getattr(_lib, f"orc_coo_to_csr_{sfx}").restype = i64
+            ft = ctypes.c_double if sfx == "f64" else ctypes.c_float
+            getattr(_lib, f"orc_laplacian_assemble_{sfx}").argtypes = [i32, P, P, P, P, ft, P]
+            getattr(_lib, f"orc_laplacian_grad_values_{sfx}").argtypes = [i32, P, P, i64, P, P, P, P,
+                                                                          P, P, P, i32]
+        _lib.orc_edge_slots.argtypes = [i32, P, P, i64, P, P, P, P, P, P]
+        _lib.orc_edge_slots.restype = i32
         _lib.orc_transpose_pattern.argtypes = [i32, i32, P, P, P, P, P]
         _lib.orc_coo_order.argtypes = [i32, i32, i64, P, P, P]
         _lib.orc_csr_check.argtypes = [i32, i32, i64, P, P, i32, P]
@@ -235,6 +241,77 @@ def diag_positions(rowptr, colind) -> np.ndarray:
     d = np.zeros(rowptr.shape[0] - 1, np.int32)
     _L().orc_diag_positions(rowptr.shape[0] - 1, _p(rowptr), _p(colind), _p(d))
     return d
+
+
+@dataclass
+class EdgeSlots:
+    code: int               # 0, or the failure code documented in oracle.c
+    where: int              # offending edge (or row, code 5); -1 when valid
+    slot_ij: np.ndarray     # int64 [E]: position of entry (i, j)
+    slot_ji: np.ndarray     # int64 [E]: position of entry (j, i)
+    owner: np.ndarray       # int64 [nnz]: edge carried by each entry, -1 for none
+
+
+def edge_slots(rowptr, colind, ei, ej) -> EdgeSlots:
+    """Pattern positions of undirected edges (see orc_edge_slots)."""
+    rowptr, colind, ei, ej = _i32(rowptr), _i32(colind), _i32(ei), _i32(ej)
+    E = ei.shape[0]
+    sij, sji = np.zeros(max(E, 1), np.int64), np.zeros(max(E, 1), np.int64)
+    owner = np.zeros(max(colind.shape[0], 1), np.int64)
+    where = np.zeros(1, np.int64)
+    code = _L().orc_edge_slots(rowptr.shape[0] - 1, _p(rowptr), _p(colind), E, _p(ei), _p(ej),
+                               _p(sij), _p(sji), _p(owner), _p(where))
+    return EdgeSlots(int(code), int(where[0]), sij[:E], sji[:E], owner[:colind.shape[0]])
+
+
+def _shifts(shift, B, dt):
+    s = np.zeros(B, dt) if shift is None else np.broadcast_to(np.asarray(shift, dt), (B,))
+    return [dt.type(v) for v in s]
+
+
+def laplacian_assemble(rowptr, colind, ei, ej, w, shift=None) -> np.ndarray:
+    """Values of L_w + shift*I on the pattern; w [E] or [B][E], shift scalar or [B]."""
+    rowptr, colind = _i32(rowptr), _i32(colind)
+    es = edge_slots(rowptr, colind, ei, ej)
+    if es.code != 0:
+        raise ValueError(f"invalid edges: code {es.code} at {es.where}")
+    dt = np.asarray(w).dtype
+    W, single = _batch(w, dt)
+    f = getattr(_L(), f"orc_laplacian_assemble_{_sfx(dt)}")
+    V = np.zeros((W.shape[0], colind.shape[0]), dt)
+    for s, sh in enumerate(_shifts(shift, W.shape[0], np.dtype(dt))):
+        vb = np.zeros(max(colind.shape[0], 1), dt)
+        f(rowptr.shape[0] - 1, _p(rowptr), _p(colind), _p(es.owner if es.owner.size else
+                                                        np.zeros(1, np.int64)),
+          _p(np.ascontiguousarray(W[s])), sh, _p(vb))
+        V[s] = vb[:colind.shape[0]]
+    return V[0] if single else V
+
+
+def laplacian_grad_values(rowptr, colind, ei, ej, G, dw=None, dshift=None):
+    """Chain rule through laplacian_assemble: returns (dL/dw [.., E], dL/dshift [..]).
+    With dw / dshift given, the results are added to copies of them."""
+    rowptr, colind, ei, ej = _i32(rowptr), _i32(colind), _i32(ei), _i32(ej)
+    es = edge_slots(rowptr, colind, ei, ej)
+    if es.code != 0:
+        raise ValueError(f"invalid edges: code {es.code} at {es.where}")
+    dt = np.asarray(G).dtype
+    Gb, single = _batch(G, dt)
+    B, E = Gb.shape[0], ei.shape[0]
+    acc = dw is not None
+    DW = _batch(dw, dt)[0].copy() if acc else np.zeros((B, E), dt)
+    DS = np.broadcast_to(np.asarray(dshift, dt), (B,)).copy() if dshift is not None else np.zeros(B, dt)
+    f = getattr(_L(), f"orc_laplacian_grad_values_{_sfx(dt)}")
+    for s in range(B):
+        dws = np.ascontiguousarray(DW[s]) if E else np.zeros(1, dt)
+        dss = np.array([DS[s]], dt)
+        f(rowptr.shape[0] - 1, _p(rowptr), _p(colind), E, _p(ei if E else np.zeros(1, np.int32)),
+          _p(ej if E else np.zeros(1, np.int32)), _p(es.slot_ij if E else np.zeros(1, np.int64)),
+          _p(es.slot_ji if E else np.zeros(1, np.int64)), _p(np.ascontiguousarray(Gb[s])), _p(dws),
+          _p(dss), int(acc or dshift is not None))
+        DW[s] = dws[:E]
+        DS[s] = dss[0]
+    return (DW[0], DS[0]) if single else (DW, DS)
 
 
 def dense_lu_solve(a, b) -> np.ndarray:

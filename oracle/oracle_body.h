@@ -201,6 +201,63 @@ int32_t FN(orc_cg_adjoint)(int32_t n, const int32_t *rowptr, const int32_t *coli
     return rc;
 }
 
+/*
+ * Edge-weighted graph Laplacian plus a diagonal shift, written into the values
+ * of a given pattern (the conductivity-to-matrix map of inverse coefficient
+ * learning, torch-sla summary page, "Experimental results", end-to-end
+ * application; the pages leave the assembly open, so this is the plain
+ * graph-Laplacian reading):
+ *   A_ij = A_ji = -w_e for every edge e = (i, j);
+ *   A_ii = (the weights of the edges at i, added one by one from 0 in
+ *           ascending neighbour index) + shift;
+ *   every other stored entry 0.
+ * owner[] is orc_edge_slots' (rows hold strictly increasing columns, so a row
+ * walk in stored order visits the neighbours in ascending index).
+ */
+void FN(orc_laplacian_assemble)(int32_t n, const int32_t *rowptr, const int32_t *colind,
+                                const int64_t *owner, const T *w, T shift, T *vals)
+{
+    for (int32_t i = 0; i < n; ++i) {
+        T d = (T)0;
+        int64_t dpos = -1;
+        for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t) {
+            if (colind[t] == i) {
+                dpos = t;
+            } else if (owner[t] >= 0) {
+                vals[t] = -w[owner[t]];
+                d = d + w[owner[t]];
+            } else {
+                vals[t] = (T)0;
+            }
+        }
+        if (dpos >= 0) vals[dpos] = d + shift;
+    }
+}
+
+/*
+ * Chain rule through orc_laplacian_assemble: with G = dL/dvals,
+ *   dL/dw_e = G_ii + G_jj - G_ij - G_ji   (added left to right),
+ *   dL/dshift = sum_i G_ii                (accumulated in double, rounded to T).
+ * With accumulate != 0 both are added to dw / *dshift instead of stored.
+ */
+void FN(orc_laplacian_grad_values)(int32_t n, const int32_t *rowptr, const int32_t *colind,
+                                   int64_t n_edges, const int32_t *ei, const int32_t *ej,
+                                   const int64_t *slot_ij, const int64_t *slot_ji,
+                                   const T *G, T *dw, T *dshift, int32_t accumulate)
+{
+    int32_t *dpos = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+    if (!dpos) return;
+    orc_diag_positions(n, rowptr, colind, dpos);
+    for (int64_t e = 0; e < n_edges; ++e) {
+        const T v = ((G[dpos[ei[e]]] + G[dpos[ej[e]]]) - G[slot_ij[e]]) - G[slot_ji[e]];
+        dw[e] = accumulate ? dw[e] + v : v;
+    }
+    double s = 0.0;
+    for (int32_t i = 0; i < n; ++i) s = s + (double)G[dpos[i]];
+    *dshift = accumulate ? *dshift + (T)s : (T)s;
+    free(dpos);
+}
+
 
 /*
  * CSR from coordinate (COO) entries: entries are ordered by (row, col) with a
