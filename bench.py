@@ -51,6 +51,18 @@ def grad_bytes(n: int, nnz: int, vbytes: int) -> int:
     return (4 + vbytes) * nnz + (2 * vbytes + 4) * n
 
 
+def edge_metrics(n: int, nnz: int, E: int, B: int, vbytes: int, asm_ms: float, grad_ms: float):
+    """Algorithmic bytes of the edge kernels: assembly reads the shared pattern
+    (row pointers, columns, entry-to-edge map) once and per system the weights,
+    writing the values; the fused gradient reads the edge list once and per
+    system lambda and x, writing dL/dw (the shift gradient's sum is included)."""
+    asm_bytes = 4 * (n + 1) + 8 * nnz + B * vbytes * (E + nnz + 1)
+    grad_bytes_ = 8 * E + B * vbytes * (2 * n + E + 1)
+    return {"assemble_ms": asm_ms, "assemble_gbs": asm_bytes / (asm_ms / 1000.0) / 1e9,
+            "assemble_bytes": asm_bytes, "edge_grad_bytes": grad_bytes_,
+            "edge_grad_gbs": grad_bytes_ / (grad_ms / 1000.0) / 1e9}
+
+
 def source_digest() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_sparse_linear_csr_b200", "csrc")
@@ -156,9 +168,10 @@ def load_workload(name: str, rank: int = 0):
     return _WORKLOAD[key]
 
 
-def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2"):
+def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2", edges: bool = False):
     """Oracle on a bounded sample of the step: k forward + k adjoint iterations +
-    gradient, on system 0 of the workload."""
+    gradient, on system 0 of the workload (with edges: assembly from the edge
+    weights first and the chain rule to them last)."""
     import numpy as np
     from oracle import oracle as O
     w = load_workload(name)
@@ -166,9 +179,14 @@ def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2"):
     v, b, xs = w.values[0].astype(npdt), w.b[0].astype(npdt), w.xstar[0].astype(npdt)
     O.build()
     t0 = time.perf_counter()
+    if edges:
+        v = O.laplacian_assemble(w.rowptr, w.colind, w.edges[0], w.edges[1],
+                                 w.weights[0].astype(npdt), w.shift)
     x, _ = O.pcg(w.rowptr, w.colind, v, b, fixed_iters=k_iters)
     lam, _ = O.cg_adjoint(w.rowptr, w.colind, v, (x - xs).astype(npdt), fixed_iters=k_iters)
-    O.grad_values(w.rowptr, w.colind, lam, x)
+    G = O.grad_values(w.rowptr, w.colind, lam, x)
+    if edges:
+        O.laplacian_grad_values(w.rowptr, w.colind, w.edges[0], w.edges[1], G)
     dt = time.perf_counter() - t0
     return 2 * k_iters / dt, dt
 
@@ -195,10 +213,10 @@ def run_reference(args):
         return 0
     k = args.ref_iters
     for _ in range(args.warmup):
-        oracle_sample(args.dtype, k, args.workload)
+        oracle_sample(args.dtype, k, args.workload, args.edges)
     total_it, total_t = 0, 0.0
     for _ in range(args.steps):
-        _, dt = oracle_sample(args.dtype, k, args.workload)
+        _, dt = oracle_sample(args.dtype, k, args.workload, args.edges)
         total_it += 2 * k
         total_t += dt
     v = total_it / total_t
@@ -209,7 +227,8 @@ def run_reference(args):
             "config": workload_config(args),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"each step: {k} forward + {k} adjoint PCG iterations + "
-                                       f"value gradient of system 0 of workload {args.workload}"},
+                                       f"{'edge-weight' if args.edges else 'value'} gradient of "
+                                       f"system 0 of workload {args.workload}"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -221,7 +240,12 @@ def workload_config(args, w=None):
         w = load_workload(args.workload)
     mode = (f"fixed {w.fixed_iters} forward + {w.fixed_iters} adjoint" if w.fixed_iters
             else f"forward and adjoint to relative residual {w.rtol:g}")
-    return {"workload": f"{w.description}: {mode} Jacobi-PCG iterations + sparse value gradient",
+    if args.edges:
+        what = (f"{w.description}: assembly from the {len(w.edges[0])} edge weights, {mode} "
+                f"Jacobi-PCG iterations, gradient to the edge weights and the shift")
+    else:
+        what = f"{w.description}: {mode} Jacobi-PCG iterations + sparse value gradient"
+    return {"workload": what, "edges": bool(args.edges),
             "name": args.workload, "n": int(w.n), "nnz": int(w.nnz), "batch": int(w.batch),
             "value_dtype": args.dtype, "l2": "flushed between steps (write of a 256 MiB buffer)",
             "parallelism": f"replicas x{world}"}
@@ -242,7 +266,12 @@ def main():
     ap.add_argument("--iters", type=int, default=0,
                     help="override the fixed iteration count (short profiler captures)")
     ap.add_argument("--workload", default="c2", choices=WORKLOADS)
+    ap.add_argument("--edges", action="store_true",
+                    help="edge-weighted workloads (c3, c4, c5, c5rcm): assemble the values from "
+                         "the edge weights and take the gradient back to them")
     args = ap.parse_args()
+    if args.edges and args.workload not in ("c3", "c4", "c5", "c5rcm"):
+        ap.error("--edges needs an edge-weighted workload (c3, c4, c5, c5rcm)")
     if args.impl == "reference":
         return run_reference(args)
 
@@ -284,17 +313,32 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    if args.edges:
+        E = len(w.edges[0])
+        Ed = sla.EdgeLaplacian(A, torch.from_numpy(w.edges[0].astype(np.int32)).to(dev),
+                               torch.from_numpy(w.edges[1].astype(np.int32)).to(dev))
+        wts = torch.from_numpy(w.weights).to(dev, dt).contiguous()
+        shift_t = torch.full((B,), w.shift, dtype=dt, device=dev)
+        dwt = torch.empty(B, E, dtype=dt, device=dev)
+        dst = torch.empty(B, dtype=dt, device=dev)
+        ews = torch.empty(max(L.sla_edges_workspace_bytes(Ed.plan), 1), dtype=torch.uint8, device=dev)
 
     def step(e=None):
         if e: e[0].record(stream)
-        L.sla_cg_solve(A.handle, vals, b, x, opts, L.make_info(*finfo), ws)
+        if args.edges:
+            L.sla_laplacian_assemble(Ed.plan, wts, shift_t, vals)
         if e: e[1].record(stream)
-        torch.sub(x, xs, out=g)                       # dL/dx of L = 0.5 ||x - x*||^2
+        L.sla_cg_solve(A.handle, vals, b, x, opts, L.make_info(*finfo), ws)
         if e: e[2].record(stream)
-        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, L.make_info(*ainfo), ws)
+        torch.sub(x, xs, out=g)                       # dL/dx of L = 0.5 ||x - x*||^2
         if e: e[3].record(stream)
-        L.sla_grad_values(A.handle, lam, x, G, 0)
+        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, L.make_info(*ainfo), ws)
         if e: e[4].record(stream)
+        if args.edges:
+            L.sla_laplacian_grad(Ed.plan, lam, x, dwt, dst, 0, ews)
+        else:
+            L.sla_grad_values(A.handle, lam, x, G, 0)
+        if e: e[5].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -304,7 +348,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local) if rank == 0 else None
-    events = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    events = [[ev() for _ in range(6)] for _ in range(args.steps)]
     for k in range(args.steps):
         flush.zero_()                                  # L2 flush, outside the step's events
         step(events[k])
@@ -313,10 +357,11 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [e[0].elapsed_time(e[4]) for e in events]
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
-    adj_ms = [e[2].elapsed_time(e[3]) for e in events]
-    grad_ms = [e[3].elapsed_time(e[4]) for e in events]
+    step_ms = [e[0].elapsed_time(e[5]) for e in events]
+    asm_ms = [e[0].elapsed_time(e[1]) for e in events]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in events]
+    adj_ms = [e[3].elapsed_time(e[4]) for e in events]
+    grad_ms = [e[4].elapsed_time(e[5]) for e in events]
     # every step does the same work (deterministic solver): iterations of the last one
     fwd_it = int(finfo[0].sum().item())
     adj_it = int(ainfo[0].sum().item())
@@ -328,10 +373,11 @@ def main():
     # ---- end to end through the public API, host buffers, loss read back
     e2e = None
     if not args.no_e2e:
-        vh = torch.from_numpy(w.values).to(dt).pin_memory()
+        # the step's inputs: the values (or the edge weights), b and x*
+        vh = torch.from_numpy(w.weights if args.edges else w.values).to(dt).pin_memory()
         bh = torch.from_numpy(w.b).to(dt).pin_memory()
         xh = torch.from_numpy(w.xstar).to(dt).pin_memory()
-        vd = torch.empty_like(vals)
+        vd = torch.empty(vh.shape, dtype=dt, device=dev)
         bd = torch.empty_like(b)
         xd = torch.empty_like(xs)
 
@@ -340,7 +386,10 @@ def main():
             bd.copy_(bh, non_blocking=True)
             xd.copy_(xh, non_blocking=True)
             vv = vd.requires_grad_(True)
-            xx = A.solve(vv, bd, rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
+            if args.edges:
+                xx = Ed.solve(vv, bd, w.shift, rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
+            else:
+                xx = A.solve(vv, bd, rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
             loss = 0.5 * ((xx - xd) ** 2).sum()
             loss.backward()
             vv.grad = None
@@ -380,6 +429,9 @@ def main():
                                               (args.strategy == 0 and props.block_fits))
         # per solve: the solver kernel (+ the sliced-value gather); then the gradient
         launches_per_step = 2 * (1 + (1 if (uses_grid and props.sliced) else 0)) + 1
+        if args.edges:
+            # assembly; the edge gradient (per edge) and the shift gradient (tile sums, finish)
+            launches_per_step += 1 + 2
         if uses_cluster:
             variant = "thread-block cluster per system, DSMEM"
         elif not uses_grid:
@@ -402,9 +454,10 @@ def main():
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             k = args.cpu_iters if args.cpu_iters > 0 else CPU_ITERS[args.workload]
-            v_cpu, t_cpu = oracle_sample(args.dtype, k, args.workload)
+            v_cpu, t_cpu = oracle_sample(args.dtype, k, args.workload, args.edges)
             cpu = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
-                   "sample": f"{k} forward + {k} adjoint PCG iterations + value gradient of "
+                   "sample": f"{k} forward + {k} adjoint PCG iterations + "
+                             f"{'assembly and edge-weight' if args.edges else 'value'} gradient of "
                              f"system 0, single-threaded C ({t_cpu:.1f} s)"}
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
@@ -415,7 +468,9 @@ def main():
                 "forward_ms": statistics.mean(fwd_ms), "adjoint_ms": statistics.mean(adj_ms),
                 "grad_ms": statistics.mean(grad_ms),
                 "forward_iters": fwd_it, "adjoint_iters": adj_it, "statuses": statuses,
-                "grad_gbs": gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
+                "grad_gbs": None if args.edges else gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
+                **(edge_metrics(n, nnz, len(w.edges[0]), B, vbytes, statistics.mean(asm_ms),
+                                statistics.mean(grad_ms)) if args.edges else {}),
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clock_info}

@@ -75,6 +75,12 @@ _SIGNATURES = {
     "sla_csr_check": ([_I32, _I32, _I64, _P, _P, _I32, _P, _P], _I32),
     "sla_cg_solve_noalloc": ([_I32, _I64, _P, _P, _I32, _I32, _P, _P, _P, ctypes.POINTER(sla_cg_opts),
                               sla_cg_info, _P], _I32),
+    "sla_edges_create": ([_P, _I64, _P, _P, ctypes.POINTER(_I64), _P, ctypes.POINTER(_P)], _I32),
+    "sla_edges_destroy": ([_P], _I32),
+    "sla_laplacian_assemble": ([_P, _P, _P, _P, _P], _I32),
+    "sla_edges_workspace_bytes": ([_P], _SZ),
+    "sla_laplacian_grad_values": ([_P, _P, _P, _P, _I32, _P, _SZ, _P], _I32),
+    "sla_laplacian_grad": ([_P, _P, _P, _P, _P, _I32, _P, _SZ, _P], _I32),
     "sla_last_error_string": ([], ctypes.c_char_p),
     "sla_version": ([], ctypes.c_char_p),
 }
@@ -235,3 +241,49 @@ def sla_cg_solve_noalloc(n, nnz, rowptr, colind, batch, dtype, vals, b, x, opts,
     _check("sla_cg_solve_noalloc", lib().sla_cg_solve_noalloc(
         n, nnz, _ptr(rowptr), _ptr(colind), batch, dtype, _ptr(vals), _ptr(b), _ptr(x),
         ctypes.byref(opts), info, _stream(stream)))
+
+
+class EdgeCheckError(SlaError):
+    """Invalid edge list: ``code`` and ``index`` as documented in include/sla.h."""
+    def __init__(self, fn: str, status: int, msg: str, check: int):
+        super().__init__(fn, status, msg)
+        self.code = check >> 40
+        self.index = check & ((1 << 40) - 1)
+
+
+def sla_edges_create(h, n_edges, ei, ej, stream=None) -> int:
+    out = _P()
+    check = _I64(0)
+    st = lib().sla_edges_create(h, n_edges, _ptr(ei), _ptr(ej), ctypes.byref(check), _stream(stream),
+                                ctypes.byref(out))
+    if st != SLA_OK:
+        msg = lib().sla_last_error_string().decode()
+        if check.value:
+            raise EdgeCheckError("sla_edges_create", st, msg, check.value)
+        raise SlaError("sla_edges_create", st, msg)
+    return out.value
+
+
+def sla_edges_destroy(e) -> None:
+    _check("sla_edges_destroy", lib().sla_edges_destroy(e))
+
+
+def sla_laplacian_assemble(e, w, shift, vals, stream=None) -> None:
+    _check("sla_laplacian_assemble", lib().sla_laplacian_assemble(e, _ptr(w), _ptr(shift), _ptr(vals),
+                                                                  _stream(stream)))
+
+
+def sla_edges_workspace_bytes(e) -> int:
+    return int(lib().sla_edges_workspace_bytes(e))
+
+
+def sla_laplacian_grad_values(e, G, dw, dshift, accumulate, ws, stream=None) -> None:
+    _check("sla_laplacian_grad_values", lib().sla_laplacian_grad_values(
+        e, _ptr(G), _ptr(dw), _ptr(dshift), int(accumulate), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sla_laplacian_grad(e, lam, x, dw, dshift, accumulate, ws, stream=None) -> None:
+    _check("sla_laplacian_grad", lib().sla_laplacian_grad(
+        e, _ptr(lam), _ptr(x), _ptr(dw), _ptr(dshift), int(accumulate), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))

@@ -14,6 +14,7 @@ the computation runs in libsla.so's kernels (see _lib.py).
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass
 
 import torch
@@ -188,3 +189,149 @@ class _Solve(torch.autograd.Function):
         gv = A.grad_values(lam, x).reshape(values.shape) if ctx.needs_input_grad[1] else None
         gb = lam.reshape(gx.shape) if ctx.needs_input_grad[2] else None
         return None, gv, gb, None
+
+
+class EdgeLaplacian:
+    """A = L_w + diag(shift) on the pattern of ``A``: the map from edge
+    conductivities to matrix values of inverse coefficient learning ("torch-sla",
+    technical summary, "Experimental results", end-to-end application).
+
+    For undirected edges e = (ei[e], ej[e]) (int32 [E] device tensors, each pair
+    once, both entries and every diagonal stored in the pattern):
+    A_ij = A_ji = -w_e and A_ii = (i's edge weights, ascending neighbour index)
+    + shift.  ``assemble`` and ``solve`` are differentiable in w, shift (and b);
+    ``solve`` assembles, solves, and in its backward runs one adjoint solve and
+    the fused edge-gradient kernel, never forming dL/dvalues.
+    """
+
+    def __init__(self, A: CSR, ei: torch.Tensor, ej: torch.Tensor):
+        self.A = A
+        self.ei = ei.to(device=A.device, dtype=torch.int32).contiguous()
+        self.ej = ej.to(device=A.device, dtype=torch.int32).contiguous()
+        self.n_edges = self.ei.numel()
+        if self.ej.numel() != self.n_edges:
+            raise ValueError("ei and ej must have the same length")
+        with torch.cuda.device(A.device):
+            self.plan = L.sla_edges_create(A.handle, self.n_edges, self.ei, self.ej)
+
+    def __del__(self):
+        p = getattr(self, "plan", None)
+        if p:
+            try:
+                torch.cuda.synchronize(self.A.device)
+                L.sla_edges_destroy(p)
+            except Exception:
+                pass
+            self.plan = None
+
+    def _w(self, w: torch.Tensor) -> torch.Tensor:
+        A = self.A
+        v = w.reshape(A.batch, self.n_edges)
+        if v.dtype != A.dtype or v.device != A.device:
+            raise TypeError(f"weights must be {A.dtype} on {A.device}")
+        return v.contiguous()
+
+    def _shift(self, shift):
+        A = self.A
+        if shift is None:
+            return None
+        if not torch.is_tensor(shift):
+            return torch.full((A.batch,), float(shift), dtype=A.dtype, device=A.device)
+        s = shift.reshape(-1)
+        if s.numel() == 1 and A.batch > 1:
+            s = s.expand(A.batch)
+        if s.dtype != A.dtype or s.device != A.device:
+            raise TypeError(f"shift must be {A.dtype} on {A.device}")
+        return s.contiguous()
+
+    # -------------------------------------------------------- primitives
+    def assemble_values(self, w, shift=None) -> torch.Tensor:
+        """values [B, nnz] of L_w + shift I, without autograd."""
+        A = self.A
+        vals = torch.empty(A.batch, A.nnz, dtype=A.dtype, device=A.device)
+        L.sla_laplacian_assemble(self.plan, self._w(w), self._shift(shift), vals)
+        return vals
+
+    def _grads(self, fn, args, dw, dshift, accumulate):
+        A = self.A
+        dw = dw if dw is not None else torch.empty(A.batch, self.n_edges, dtype=A.dtype, device=A.device)
+        ws = _workspace(L.sla_edges_workspace_bytes(self.plan), A.device) if dshift is not None else None
+        fn(self.plan, *args, dw, dshift, int(accumulate), ws)
+        return dw, dshift
+
+    def grad_from_values(self, G, dw=None, dshift=None, accumulate=False, want_shift=True):
+        """(dL/dw [B, E], dL/dshift [B]) from G = dL/dvalues by the chain rule."""
+        A = self.A
+        if dshift is None and want_shift:
+            dshift = torch.empty(A.batch, dtype=A.dtype, device=A.device)
+        return self._grads(L.sla_laplacian_grad_values, (A._values(G),), dw, dshift, accumulate)
+
+    def grad(self, lam, x, dw=None, dshift=None, accumulate=False, want_shift=True):
+        """The same for G = -lam x^T on the pattern, without forming G."""
+        A = self.A
+        if dshift is None and want_shift:
+            dshift = torch.empty(A.batch, dtype=A.dtype, device=A.device)
+        return self._grads(L.sla_laplacian_grad, (A._vec(lam, A.n_rows), A._vec(x, A.n_rows)),
+                           dw, dshift, accumulate)
+
+    # ---------------------------------------------------- autograd calls
+    def assemble(self, w, shift=None) -> torch.Tensor:
+        """values = L_w + shift I, differentiable in w and shift."""
+        return _Assemble.apply(self, w, shift)
+
+    def solve(self, w, b, shift=None, *, rtol=1e-10, atol=0.0, max_iter=0, fixed_iters=0,
+              precond=True, strategy=L.SLA_STRATEGY_AUTO) -> torch.Tensor:
+        """x = (L_w + shift I)^-1 b, differentiable in w, shift and b."""
+        opts = dict(rtol=rtol, atol=atol, max_iter=max_iter, fixed_iters=fixed_iters,
+                    precond=precond, strategy=strategy)
+        return _EdgeSolve.apply(self, w, shift, b, opts)
+
+
+class _Assemble(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, E: EdgeLaplacian, w, shift):
+        ctx.E = E
+        ctx.shift_shape = None if shift is None or not torch.is_tensor(shift) else shift.shape
+        return E.assemble_values(w, shift).reshape(w.shape[:-1] + (E.A.nnz,))
+
+    @staticmethod
+    def backward(ctx, gv):
+        E = ctx.E
+        want_s = ctx.needs_input_grad[2]
+        dw, ds = E.grad_from_values(gv.contiguous(), want_shift=want_s)
+        gw = dw.reshape(gv.shape[:-1] + (E.n_edges,)) if ctx.needs_input_grad[1] else None
+        gs = ds.reshape(ctx.shift_shape) if want_s and ds.numel() == math.prod(ctx.shift_shape) else \
+            (ds.sum().reshape(ctx.shift_shape) if want_s else None)
+        return None, gw, gs
+
+
+class _EdgeSolve(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, E: EdgeLaplacian, w, shift, b, opts):
+        A = E.A
+        vals = E.assemble_values(w, shift)
+        x, info = A.cg(vals, b, **opts)
+        A.last_info = info
+        ctx.E, ctx.opts = E, opts
+        ctx.shift_shape = None if shift is None or not torch.is_tensor(shift) else shift.shape
+        ctx.w_shape = w.shape
+        ctx.save_for_backward(vals, x)
+        return x.reshape(b.shape)
+
+    @staticmethod
+    def backward(ctx, gx):
+        E, opts = ctx.E, ctx.opts
+        A = E.A
+        vals, x = ctx.saved_tensors
+        lam, info = A.cg(vals, gx.contiguous(), adjoint=True, **opts)
+        A.last_adjoint_info = info
+        want_s = ctx.needs_input_grad[2]
+        gw = gs = None
+        if ctx.needs_input_grad[1] or want_s:
+            dw, ds = E.grad(lam, x, want_shift=want_s)
+            gw = dw.reshape(ctx.w_shape) if ctx.needs_input_grad[1] else None
+            if want_s:
+                gs = ds.reshape(ctx.shift_shape) if ds.numel() == math.prod(ctx.shift_shape) else \
+                    ds.sum().reshape(ctx.shift_shape)
+        gb = lam.reshape(gx.shape) if ctx.needs_input_grad[3] else None
+        return None, gw, gs, gb, None

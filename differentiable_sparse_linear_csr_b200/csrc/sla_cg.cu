@@ -549,7 +549,6 @@ cg_grid2_kernel(CgArgs<T> a) {
     __shared__ double red[4 * 33];
     __shared__ int flag;
     const int tid = threadIdx.x;
-    const int G = gridDim.x;
     const int n = a.n;
     const int tile = blockIdx.x;                 // one tile per block, one system
     const bool has_tile = tile < a.ntiles;

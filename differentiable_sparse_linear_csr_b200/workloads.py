@@ -272,6 +272,11 @@ class Workload:
     rtol: float                 # relative residual target (0 when fixed_iters > 0)
     fixed_iters: int            # > 0: run exactly this many iterations
     description: str = ""
+    # edge-weighted Laplacians only: the undirected edges (ei, ej) in this
+    # workload's row numbering, their weights [B][E] and the diagonal shift
+    edges: tuple | None = None
+    weights: np.ndarray | None = None
+    shift: float = 0.0
 
     @property
     def nnz(self) -> int:
@@ -314,7 +319,8 @@ def c3_diffusion3d(seed: int = 3, N: int = 128) -> Workload:
     return Workload(f"c3_diffusion3d_{N}", n, rp, ci, _as_batch(v),
                     _as_batch(uniform(seed, STREAM_B, n, -1, 1)),
                     _as_batch(uniform(seed, STREAM_XSTAR, n, -1, 1)),
-                    1e-8, 0, f"3-D 7-point log-normal diffusion {N}^3 + 1e-3 I, PCG to 1e-8")
+                    1e-8, 0, f"3-D 7-point log-normal diffusion {N}^3 + 1e-3 I, PCG to 1e-8",
+                    (ei, ej), w[None, :], 1e-3)
 
 
 def c4_batched(seed: int = 4, B: int = 1024, N: int = 32) -> Workload:
@@ -326,7 +332,8 @@ def c4_batched(seed: int = 4, B: int = 1024, N: int = 32) -> Workload:
     return Workload(f"c4_batched_{B}x{N}x{N}", n, rp, ci, _as_batch(v),
                     normal(seed, STREAM_B, B * n).reshape(B, n),
                     uniform(seed, STREAM_XSTAR, B * n, -1, 1).reshape(B, n),
-                    1e-10, 0, f"{B} shared-pattern {N}x{N} diffusion systems + 1e-2 I, PCG to 1e-10")
+                    1e-10, 0, f"{B} shared-pattern {N}x{N} diffusion systems + 1e-2 I, PCG to 1e-10",
+                    (ei, ej), w, 1e-2)
 
 
 def c5_knn(seed: int = 5, npts: int = 8_000_000, k: int = 8, order: str = "generated") -> Workload:
@@ -340,10 +347,14 @@ def c5_knn(seed: int = 5, npts: int = 8_000_000, k: int = 8, order: str = "gener
         perm = rcm_permutation(rp, ci, npts)
         rp, ci, v = permute_symmetric(rp, ci, v, perm)
         b, xs = b[perm], xs[perm]
+        inv = np.empty(npts, dtype=np.int64)
+        inv[perm] = np.arange(npts)
+        ei, ej = inv[ei], inv[ej]                 # the same edges, renumbered
     elif order != "generated":
         raise ValueError(order)
     return Workload(f"c5_knn_{npts}_{order}", npts, rp, ci, _as_batch(v), _as_batch(b), _as_batch(xs),
-                    1e-8, 0, f"{k}-NN graph Laplacian on {npts} points ({order} order) + 1e-3 I, PCG to 1e-8")
+                    1e-8, 0, f"{k}-NN graph Laplacian on {npts} points ({order} order) + 1e-3 I, PCG to 1e-8",
+                    (ei, ej), w[None, :], 1e-3)
 
 
 CONFIGS = {

@@ -299,6 +299,64 @@ sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t *rowptr,
                                 const void *vals, const void *b, void *x,
                                 const sla_cg_opts *opts, sla_cg_info info, void *stream);
 
+/*
+ * Edge-weighted graph Laplacian on a handle's pattern: the map from edge
+ * conductivities to matrix values used by inverse coefficient learning
+ * (torch-sla summary page, technical summary, "Experimental results",
+ * end-to-end application: spatially varying conductivities of a Poisson
+ * problem recovered through A.solve with a standard Adam loop).  The pages do
+ * not spell the assembly out; this is the plain graph-Laplacian reading.  For
+ * system b with weights w_b [E] and shift s_b:
+ *   A_ij = A_ji = -w_e                  for edge e = (i, j), i != j;
+ *   A_ii = (the weights of the edges at i, added one by one from 0 in
+ *           ascending neighbour index) + s_b;
+ *   every other stored entry = 0.
+ * The gradient follows by the chain rule from G = dL/dvals (for a solve,
+ * G_ij = -lambda_i x_j, "Methodology" 2):
+ *   dL/dw_e = ((G_ii + G_jj) - G_ij) - G_ji,   dL/ds_b = sum_i G_ii.
+ *
+ * sla_edges_create maps undirected edges (device int32 ei[E], ej[E], read
+ * only during the call) to their two pattern entries and keeps that map
+ * (8 E + 4 nnz bytes of device memory, owned by the plan).  The handle must be
+ * square and must outlive the plan.  It synchronises the host once.  Invalid
+ * edges give SLA_ERR_INVALID; *check (host, may be NULL) receives
+ * code << 40 | index of the failure with the smallest code, then the smallest
+ * index (0 when valid):
+ *   1 an endpoint outside [0, n)        (index: the edge)
+ *   2 a self loop, i == j               (the edge)
+ *   3 entry (i, j) or (j, i) not in the pattern   (the edge)
+ *   4 an unordered pair that an earlier edge already names   (the later edge)
+ *   5 a row without a diagonal entry    (the row)
+ */
+typedef struct sla_edges_s *sla_edges_t;
+sla_status sla_edges_create(sla_csr_t h, int64_t n_edges, const int32_t *ei, const int32_t *ej,
+                            int64_t *check, void *stream, sla_edges_t *out);
+sla_status sla_edges_destroy(sla_edges_t e);
+
+/* vals (device [B][nnz], the handle's dtype) = A(w, shift) for w (device
+ * [B][E]) and shift (device [B], or NULL for 0).  Bit-exact: each entry is
+ * one negation or the ordered sum above. */
+sla_status sla_laplacian_assemble(sla_edges_t e, const void *w, const void *shift, void *vals,
+                                  void *stream);
+
+/* Workspace (256-byte aligned) of the two gradient calls below. */
+size_t sla_edges_workspace_bytes(sla_edges_t e);
+
+/* dw (device [B][E]) and dshift (device [B], may be NULL) from G (device
+ * [B][nnz]) by the chain rule above; with accumulate != 0 they are added to
+ * dw / dshift.  dw is bit-exact (four entries added in the stated order);
+ * dshift is accumulated in double over a fixed tree and rounded once. */
+sla_status sla_laplacian_grad_values(sla_edges_t e, const void *G, void *dw, void *dshift,
+                                     int32_t accumulate, void *ws, size_t ws_bytes, void *stream);
+
+/* The same with G = -lambda x^T on the pattern (what sla_grad_values would
+ * write), without forming G: each G entry is rounded exactly as
+ * sla_grad_values rounds it, so dw equals sla_grad_values followed by
+ * sla_laplacian_grad_values bit for bit.  lambda, x: device [B][n]. */
+sla_status sla_laplacian_grad(sla_edges_t e, const void *lambda, const void *x, void *dw,
+                              void *dshift, int32_t accumulate, void *ws, size_t ws_bytes,
+                              void *stream);
+
 /* Message for the last non-OK status on this host thread ("" if none). */
 const char *sla_last_error_string(void);
 

@@ -59,6 +59,16 @@ def test_host_side_argument_errors_need_no_gpu():
     assert lib.sla_cg_adjoint(None, None, None, None, ctypes.byref(opts), info, None, 0, None) == L.SLA_ERR_INVALID
     assert lib.sla_workspace_bytes(None, L.SLA_OP_CG) == 0
     assert lib.sla_csr_destroy(None) == L.SLA_OK
+    e = ctypes.c_void_p()
+    check = ctypes.c_int64(7)
+    assert lib.sla_edges_create(None, 0, None, None, ctypes.byref(check), None,
+                                ctypes.byref(e)) == L.SLA_ERR_INVALID
+    assert e.value is None and check.value == 0 and "handle" in L.sla_last_error_string()
+    assert lib.sla_laplacian_assemble(None, None, None, None, None) == L.SLA_ERR_INVALID
+    assert lib.sla_laplacian_grad_values(None, None, None, None, 0, None, 0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_laplacian_grad(None, None, None, None, None, 0, None, 0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_edges_workspace_bytes(None) == 0
+    assert lib.sla_edges_destroy(None) == L.SLA_OK
 
 
 def test_workspace_sizes_grow_with_size():

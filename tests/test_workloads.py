@@ -79,3 +79,27 @@ def test_rcm_is_a_bandwidth_reducing_permutation():
     d1 = W.csr_to_dense(r.rowptr, r.colind, r.values[0])
     assert np.array_equal(d1, d0[np.ix_(perm, perm)])     # P A P^T, values moved not combined
     assert np.array_equal(r.b[0], w.b[0][perm])
+
+
+@pytest.mark.parametrize("make", [lambda: W.c4_batched(B=3, N=8), lambda: W.c3_diffusion3d(N=6),
+                                  lambda: W.c5_knn(npts=2000), lambda: W.c5_knn(npts=2000, order="rcm")])
+def test_edge_weighted_workloads_carry_their_edges(make):
+    """Edges, weights and shift reproduce the workload's values through the
+    oracle's assembly bit for bit.  In RCM order the workload's values are the
+    generated-order matrix permuted, whose diagonals were summed in the old
+    neighbour order, while assembly from the renumbered edges sums them in the
+    new order: off-diagonal entries still agree bit for bit, diagonals to
+    rounding."""
+    from oracle import oracle as O
+    w = make()
+    ei, ej = w.edges
+    assert ei.shape == ej.shape and w.weights.shape == (w.batch, ei.shape[0])
+    v = O.laplacian_assemble(w.rowptr, w.colind, ei, ej, w.weights, w.shift).reshape(w.values.shape)
+    if "rcm" not in w.name:
+        assert np.array_equal(v.view(np.uint64), w.values.view(np.uint64))
+        return
+    d = O.diag_positions(w.rowptr, w.colind)
+    off = np.ones(w.nnz, bool)
+    off[d] = False
+    assert np.array_equal(v[:, off], w.values[:, off])
+    assert np.all(np.abs(v[:, d] - w.values[:, d]) <= 32 * 2.0 ** -52 * np.abs(w.values[:, d]))
