@@ -431,7 +431,9 @@ def test_adjoint_memory_does_not_grow_with_iterations():
 
 # ------------------------------------------------------------ edge cases ----
 
-def test_edge_cases_match_oracle_outcomes():
+@pytest.mark.parametrize("onchip", ["1", "3"])
+def test_edge_cases_match_oracle_outcomes(onchip, monkeypatch):
+    _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.random_spd(300, 0.02, 4)
     A = make(rp, ci)
     b = W.uniform(4, 0, 300, -1, 1)
