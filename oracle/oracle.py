@@ -321,3 +321,42 @@ def dense_lu_solve(a, b) -> np.ndarray:
     if _L().orc_dense_lu_solve(a.shape[0], _p(a), _p(x)) != 0:
         raise np.linalg.LinAlgError("singular matrix")
     return x
+
+
+@dataclass
+class NewtonInfo:
+    steps: int                  # Newton steps taken
+    residual_norms: list        # ||F(u_k)||_2 of system 0..B-1 at every step, k = 0..steps
+    converged: bool
+
+
+def newton(rowptr, colind, residual, jacobian, u0, *, tol=1e-10, max_steps=50, cg_rtol=1e-13):
+    """Newton's method for F(u) = 0 with a sparse SPD Jacobian on the pattern
+    (nonlinear systems of torch-sla, technical summary, "Methodology" 2): the
+    plain iteration u <- u - J(u)^-1 F(u), each linear solve by the oracle's
+    PCG.  residual(u) -> F [B][n] and jacobian(u) -> values [B][nnz] are numpy
+    callables; stops when every system has ||F(u)|| <= tol * max(1, ||F(u0)||)."""
+    u = np.array(u0, dtype=np.float64, copy=True)
+    single = u.ndim == 1
+    U = u[None, :] if single else u
+    F = np.atleast_2d(residual(U))
+    norms = [np.linalg.norm(F, axis=1)]
+    bound = tol * np.maximum(1.0, norms[0])
+    steps = 0
+    while not np.all(norms[-1] <= bound) and steps < max_steps:
+        Jv = np.atleast_2d(jacobian(U))
+        delta, _ = pcg(rowptr, colind, Jv, F, rtol=cg_rtol)
+        U = U - np.atleast_2d(delta)
+        F = np.atleast_2d(residual(U))
+        norms.append(np.linalg.norm(F, axis=1))
+        steps += 1
+    info = NewtonInfo(steps, [n.tolist() for n in norms], bool(np.all(norms[-1] <= bound)))
+    return (U[0] if single else U), info
+
+
+def newton_adjoint(rowptr, colind, jac_values, gu, *, cg_rtol=1e-13):
+    """The adjoint of F(u, theta) = 0 at its solution: J^T lambda = dL/du (one
+    oracle adjoint solve); then dL/dtheta = -lambda^T dF/dtheta is the caller's
+    vector-Jacobian product with -lambda."""
+    lam, _ = cg_adjoint(rowptr, colind, jac_values, gu, rtol=cg_rtol)
+    return lam
