@@ -335,3 +335,80 @@ class _EdgeSolve(torch.autograd.Function):
                     ds.sum().reshape(ctx.shift_shape)
         gb = lam.reshape(gx.shape) if ctx.needs_input_grad[3] else None
         return None, gw, gs, gb, None
+
+
+@dataclass
+class NewtonInfo:
+    """Outcome of newton_solve (host values; each Newton step reads ||F||)."""
+    steps: int
+    residual_norms: list        # per step, the per-system ||F(u_k)||_2
+    converged: bool
+    linear: list                # per step, (iterations, statuses) of its linear solve
+
+
+def newton_solve(A: CSR, residual, jacobian, u0, *theta, tol=1e-10, max_steps=50, cg_rtol=1e-12,
+                 max_iter=0, precond=True, strategy=L.SLA_STRATEGY_AUTO) -> torch.Tensor:
+    """u with F(u, theta) = 0 by Newton's method, differentiable in theta.
+
+    Nonlinear systems of "torch-sla" (technical summary, "Methodology" 2): the
+    Jacobian J = dF/du must be SPD with A's pattern (each Newton step is one
+    Jacobi-PCG solve J delta = F, u <- u - delta); the backward pass is one
+    adjoint solve J(u)^T lambda = dL/du and one vector-Jacobian product,
+    dL/dtheta = -lambda^T dF/dtheta, whatever the number of Newton steps.
+
+    theta are tensors; residual(u, *theta) -> F shaped like u (differentiable in
+    theta, torch);
+    jacobian(u, *theta) -> J's values [B, nnz] on A's pattern.  Stops when
+    every system has ||F|| <= tol * max(1, ||F(u0)||).  A.last_newton_info
+    holds the NewtonInfo of the last forward.
+    """
+    opts = dict(tol=tol, max_steps=max_steps, cg=dict(rtol=cg_rtol, max_iter=max_iter,
+                                                      precond=precond, strategy=strategy))
+    return _Newton.apply(A, residual, jacobian, opts, u0, *theta)
+
+
+class _Newton(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, A: CSR, residual, jacobian, opts, u0, *theta):
+        u = A._vec(u0, A.n_rows).clone()
+        F = A._vec(residual(u, *theta), A.n_rows)
+        # host copies only, so that nothing kept grows with the step count
+        norms = [torch.linalg.vector_norm(F, dim=1).tolist()]
+        bound = [opts["tol"] * max(1.0, v) for v in norms[0]]
+        done = lambda nr: all(v <= t for v, t in zip(nr, bound))  # noqa: E731
+        linear = []
+        steps = 0
+        while steps < opts["max_steps"] and not done(norms[-1]):
+            Jv = A._values(jacobian(u, *theta))
+            delta, info = A.cg(Jv, F, **opts["cg"])
+            linear.append((info.iters.tolist(), info.status.tolist()))
+            u.sub_(delta)
+            del Jv, delta, info
+            F = A._vec(residual(u, *theta), A.n_rows)
+            norms.append(torch.linalg.vector_norm(F, dim=1).tolist())
+            steps += 1
+        A.last_newton_info = NewtonInfo(steps, norms, done(norms[-1]), linear)
+        ctx.A, ctx.residual, ctx.jacobian, ctx.opts = A, residual, jacobian, opts
+        ctx.u_shape = u0.shape
+        ctx.save_for_backward(u, *theta)
+        return u.reshape(u0.shape)
+
+    @staticmethod
+    def backward(ctx, gu):
+        A, opts = ctx.A, ctx.opts
+        u, *theta = ctx.saved_tensors
+        needs = ctx.needs_input_grad[5:]
+        if not any(needs):
+            return (None,) * (5 + len(theta))
+        with torch.no_grad():
+            Jv = A._values(ctx.jacobian(u, *theta))
+        lam, info = A.cg(Jv, A._vec(gu.contiguous(), A.n_rows), adjoint=True, **opts["cg"])
+        A.last_adjoint_info = info
+        with torch.enable_grad():
+            th = [t.detach().requires_grad_(need) for t, need in zip(theta, needs)]
+            F = ctx.residual(u.detach().reshape(ctx.u_shape), *th)
+            wrt = [t for t, need in zip(th, needs) if need]
+            got = torch.autograd.grad(F, wrt, grad_outputs=-lam.reshape(F.shape), allow_unused=True)
+        it = iter(got)
+        grads = [next(it) if need else None for need in needs]
+        return (None, None, None, None, None, *grads)
