@@ -8,7 +8,7 @@ the edge-weighted Laplacian with its chain rule to edge weights
 adjoint (api.newton_solve).
 The CUDA library is loaded on first use and is required: there is no CPU path.
 """
-from .api import CSR, EdgeLaplacian, NewtonInfo, SolveInfo, newton_solve  # noqa: F401
+from .api import CSR, CSRList, EdgeLaplacian, NewtonInfo, SolveInfo, newton_solve  # noqa: F401
 from . import _lib  # noqa: F401
 
-__all__ = ["CSR", "EdgeLaplacian", "NewtonInfo", "SolveInfo", "newton_solve"]
+__all__ = ["CSR", "CSRList", "EdgeLaplacian", "NewtonInfo", "SolveInfo", "newton_solve"]

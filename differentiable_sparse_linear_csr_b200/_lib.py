@@ -52,7 +52,9 @@ class sla_csr_props(ctypes.Structure):
                 ("grid_blocks", ctypes.c_int32), ("block_fits", ctypes.c_int32),
                 ("has_transpose", ctypes.c_int32), ("grid_onchip", ctypes.c_int32),
                 ("grid_tile_rows", ctypes.c_int32), ("sliced", ctypes.c_int32),
-                ("block_resident", ctypes.c_int32), ("cluster_fits", ctypes.c_int32)]
+                ("block_resident", ctypes.c_int32), ("cluster_fits", ctypes.c_int32),
+                ("n_items", ctypes.c_int32), ("item_rows_max", ctypes.c_int32),
+                ("item_smem_rows", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -75,6 +77,7 @@ _SIGNATURES = {
     "sla_csr_check": ([_I32, _I32, _I64, _P, _P, _I32, _P, _P], _I32),
     "sla_cg_solve_noalloc": ([_I32, _I64, _P, _P, _I32, _I32, _P, _P, _P, ctypes.POINTER(sla_cg_opts),
                               sla_cg_info, _P], _I32),
+    "sla_csr_list_create": ([_I32, _P, _I32, _I64, _P, _P, _I32, _U32, _P, ctypes.POINTER(_P)], _I32),
     "sla_edges_create": ([_P, _I64, _P, _P, ctypes.POINTER(_I64), _P, ctypes.POINTER(_P)], _I32),
     "sla_edges_destroy": ([_P], _I32),
     "sla_laplacian_assemble": ([_P, _P, _P, _P, _P], _I32),
@@ -152,6 +155,14 @@ def sla_csr_create(n_rows, n_cols, nnz, rowptr, colind, batch, dtype, flags, str
     _check("sla_csr_create", lib().sla_csr_create(n_rows, n_cols, nnz, _ptr(rowptr), _ptr(colind),
                                                   batch, dtype, flags, _stream(stream), ctypes.byref(h)))
     return h.value
+
+
+def sla_csr_list_create(n_items, item_rows, n_rows, nnz, rowptr, colind, dtype, flags, stream=None) -> int:
+    out = _P()
+    _check("sla_csr_list_create", lib().sla_csr_list_create(
+        n_items, _ptr(item_rows), n_rows, nnz, _ptr(rowptr), _ptr(colind), dtype, flags,
+        _stream(stream), ctypes.byref(out)))
+    return out.value
 
 
 def sla_csr_destroy(h) -> None:

@@ -70,6 +70,7 @@ class CSR:
         with torch.cuda.device(self.device):
             self.handle = L.sla_csr_create(self.n_rows, self.n_cols, self.nnz, self.rowptr, self.colind,
                                            self.batch, L.dtype_code(dtype), flags)
+        self.n_info = self.batch                 # entries of a solve's SolveInfo
         self.last_info: SolveInfo | None = None
         self.last_adjoint_info: SolveInfo | None = None
 
@@ -117,7 +118,7 @@ class CSR:
         rhs = self._vec(b, self.n_rows)
         x = self._vec(x0, self.n_rows).clone() if x0 is not None else \
             torch.empty(self.batch, self.n_rows, dtype=self.dtype, device=self.device)
-        info = _new_info(self.batch, self.device)
+        info = _new_info(self.n_info, self.device)
         opts = L.make_opts(rtol, atol, max_iter, fixed_iters, precond, x0 is not None,
                            wait_timeout_ns, strategy)
         op = L.SLA_OP_ADJOINT if adjoint else L.SLA_OP_CG
@@ -147,6 +148,65 @@ class CSR:
         opts = dict(rtol=rtol, atol=atol, max_iter=max_iter, fixed_iters=fixed_iters,
                     precond=precond, strategy=strategy)
         return _Solve.apply(self, values, b, opts)
+
+
+class CSRList(CSR):
+    """Independent square systems with their own patterns (torch-sla's
+    SparseTensorList, technical summary, "Methodology" 1), held as one
+    block-diagonal CSR: item s owns rows and columns [item_rows[s],
+    item_rows[s+1]).  Values [nnz] and vectors [n_rows] are the items'
+    concatenations; ``solve`` / ``cg`` solve every item on its own (SolveInfo
+    per item), ``matvec`` and the gradients act item by item as they must for a
+    block-diagonal matrix.  Build one with ``CSRList.from_items``.
+    """
+
+    def __init__(self, item_rows: torch.Tensor, rowptr: torch.Tensor, colind: torch.Tensor,
+                 dtype: torch.dtype = torch.float64, symmetric: bool = False, validate: bool = True):
+        if rowptr.device.type != "cuda" or colind.device.type != "cuda":
+            raise ValueError("CSRList needs CUDA tensors")
+        self.rowptr = rowptr.to(torch.int32).contiguous()
+        self.colind = colind.to(torch.int32).contiguous()
+        self.item_rows = item_rows.to(device=self.rowptr.device, dtype=torch.int32).contiguous()
+        self.n_rows = self.n_cols = self.rowptr.numel() - 1
+        self.nnz = self.colind.numel()
+        self.batch = 1
+        self.n_items = self.item_rows.numel() - 1
+        self.dtype = dtype
+        self.device = self.rowptr.device
+        self.symmetric = bool(symmetric)
+        flags = (L.SLA_FLAG_VALIDATE if validate else 0) | (L.SLA_FLAG_SYMMETRIC if symmetric else 0)
+        with torch.cuda.device(self.device):
+            self.handle = L.sla_csr_list_create(self.n_items, self.item_rows, self.n_rows, self.nnz,
+                                                self.rowptr, self.colind, L.dtype_code(dtype), flags)
+        self.n_info = self.n_items
+        self.last_info = None
+        self.last_adjoint_info = None
+
+    @classmethod
+    def from_items(cls, items, dtype=torch.float64, symmetric=False, validate=True, device=None):
+        """items: sequence of (rowptr, colind) per item (local indices)."""
+        rps, cis, rows, ents = [], [], [0], [0]
+        for rp, ci in items:
+            rp = torch.as_tensor(rp, dtype=torch.int64, device=device)
+            ci = torch.as_tensor(ci, dtype=torch.int64, device=device)
+            rps.append(rp[:-1] + ents[-1])
+            cis.append(ci + rows[-1])
+            rows.append(rows[-1] + rp.numel() - 1)
+            ents.append(ents[-1] + ci.numel())
+        rowptr = torch.cat(rps + [torch.tensor([ents[-1]], dtype=torch.int64, device=rps[0].device)])
+        colind = torch.cat(cis)
+        item_rows = torch.tensor(rows, dtype=torch.int64)
+        dev = device or torch.device("cuda")
+        return cls(item_rows.to(dev), rowptr.to(dev), colind.to(dev), dtype=dtype, symmetric=symmetric,
+                   validate=validate)
+
+    def split(self, t: torch.Tensor, per: str = "rows"):
+        """Per-item views of a concatenated vector (per='rows') or of values
+        (per='entries')."""
+        bounds = self.item_rows.tolist() if per == "rows" else \
+            self.rowptr[self.item_rows.long()].tolist()
+        t = t.reshape(-1)
+        return [t[a:b] for a, b in zip(bounds[:-1], bounds[1:])]
 
 
 class _MatVec(torch.autograd.Function):

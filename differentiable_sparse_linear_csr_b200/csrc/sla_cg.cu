@@ -835,6 +835,151 @@ cg_block_kernel(CgArgs<T> a) {
     }
 }
 
+// ---------------------------------------------------- segment kernel ----
+// A list of independent systems with their own patterns, stored as one
+// block-diagonal CSR whose item s owns rows (and columns) [seg[s], seg[s+1]).
+// Each block claims items from an atomic counter, largest first (order[]),
+// and runs the whole PCG of an item itself, exactly as cg_block_kernel does for
+// one system; an item's vectors live in shared memory when it has at most
+// smem_rows rows, else in the workspace vectors at the item's offset.  An item
+// is always solved by one block, so results do not depend on the schedule.
+template <typename T, int LANES>
+__global__ void __launch_bounds__(kCgThreads)
+cg_segment_kernel(CgArgs<T> a, const int32_t *__restrict__ seg, const int32_t *__restrict__ order,
+                  int n_items, int smem_rows, unsigned *work) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ double red[72];
+    __shared__ int s_next;
+    constexpr int NSUB = kCgThreads / LANES;
+    const int tid = threadIdx.x, sub = tid / LANES, lane = tid % LANES;
+    T *sm = reinterpret_cast<T *>(smem_raw);
+    while (true) {
+        __syncthreads();
+        if (tid == 0) s_next = (int)atomicAdd(work, 1u);
+        __syncthreads();
+        const int q = s_next;
+        if (q >= n_items) break;
+        const int s = __ldg(order + q);
+        const int o = __ldg(seg + s), m = __ldg(seg + s + 1) - o;
+        const bool on_chip = m <= smem_rows;
+        T *xs = on_chip ? sm : a.x + o;
+        T *rs = on_chip ? sm + m : a.r + o;
+        T *ps = on_chip ? sm + 2 * m : a.p + o;
+        T *qs = on_chip ? sm + 3 * m : a.q + o;
+        T *ds = on_chip ? sm + 4 * m : a.d + o;
+        const T *bs = a.b + o;
+        T *xg = a.x + o;
+        // row li of the item is global row o + li; its columns are global too
+        auto spmv_row = [&](const T *v, int li) -> T {
+            const int t0 = __ldg(a.rowptr + o + li), t1 = __ldg(a.rowptr + o + li + 1);
+            T acc = T(0);
+            for (int t = t0 + lane; t < t1; t += LANES) acc += __ldg(a.vals + t) * v[__ldg(a.colind + t) - o];
+            if constexpr (LANES > 1) {
+                const unsigned mk = subwarp_mask<LANES>();
+#pragma unroll
+                for (int off = LANES / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(mk, acc, off, LANES);
+            }
+            return acc;
+        };
+        if (a.x0_given) {
+            if (on_chip) {
+                for (int i = tid; i < m; i += kCgThreads) xs[i] = xg[i];
+                __syncthreads();
+            }
+            for (int i = sub; i < m; i += NSUB) {
+                const T v = spmv_row(xs, i);
+                if (lane == 0) qs[i] = v;
+            }
+            __syncthreads();
+        }
+        double bb = 0.0, rho = 0.0, rr = 0.0, bad = 0.0;
+        for (int i = tid; i < m; i += kCgThreads) {
+            const T bi = bs[i];
+            T ri;
+            if (a.x0_given) {
+                ri = bi - qs[i];
+            } else {
+                ri = bi;
+                xs[i] = T(0);
+            }
+            T di = T(1);
+            if (a.precond) {
+                const int dp = __ldg(a.diagpos + o + i);
+                const T dv = dp >= 0 ? __ldg(a.vals + dp) : T(0);
+                if (!(dv > T(0))) bad += 1.0;
+                di = T(1) / dv;
+            }
+            const T zi = di * ri;
+            rs[i] = ri;
+            ps[i] = zi;
+            ds[i] = di;
+            bb += (double)bi * (double)bi;
+            rho += (double)ri * (double)zi;
+            rr += (double)ri * (double)ri;
+        }
+        block_sum2<kCgThreads>(bb, rho, red);
+        block_sum2<kCgThreads>(rr, bad, red);
+        const double nb = sqrt(bb);
+        const double tol = fmax(a.rtol * nb, a.atol);
+        int st = kActive, k = 0;
+        double relres = 0.0;
+        if (nb == 0.0) st = SLA_CONVERGED;
+        else if (!isfinite(nb)) st = SLA_NONFINITE;
+        else if (a.precond && bad > 0.0) { st = SLA_BREAKDOWN; relres = sqrt(rr) / nb; }
+        else if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; relres = sqrt(rr) / nb; }
+        else if (rr == 0.0) st = SLA_CONVERGED;
+        if (nb == 0.0)
+            for (int i = tid; i < m; i += kCgThreads) xs[i] = T(0);
+        __syncthreads();
+        while (st == kActive) {
+            double sg = 0.0;
+            for (int i = sub; i < m; i += NSUB) {
+                const T qi = spmv_row(ps, i);
+                if (lane == 0) {
+                    qs[i] = qi;
+                    sg += (double)ps[i] * (double)qi;
+                }
+            }
+            const double sigma = block_sum<kCgThreads>(sg, red);
+            if (!isfinite(sigma) || !(sigma > 0.0)) {
+                st = isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE;
+                relres = sqrt(rr) / nb;
+                break;
+            }
+            const T al = (T)(rho / sigma);
+            double lrho = 0.0, lrr = 0.0;
+            for (int i = tid; i < m; i += kCgThreads) {
+                xs[i] = xs[i] + al * ps[i];
+                const T ri = rs[i] - al * qs[i];
+                rs[i] = ri;
+                const T zi = ds[i] * ri;
+                lrho += (double)ri * (double)zi;
+                lrr += (double)ri * (double)ri;
+            }
+            ++k;
+            block_sum2<kCgThreads>(lrho, lrr, red);
+            rr = lrr;
+            relres = sqrt(rr) / nb;
+            if (!isfinite(rr)) { st = SLA_NONFINITE; break; }
+            if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; break; }
+            if (rr == 0.0) { st = SLA_CONVERGED; break; }
+            if (k >= a.limit) { st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED; break; }
+            const T bt = (T)(lrho / rho);
+            rho = lrho;
+            for (int i = tid; i < m; i += kCgThreads) ps[i] = ds[i] * rs[i] + bt * ps[i];
+            __syncthreads();
+        }
+        __syncthreads();
+        if (on_chip)
+            for (int i = tid; i < m; i += kCgThreads) xg[i] = xs[i];
+        if (tid == 0) {
+            if (a.out_status) a.out_status[s] = st;
+            if (a.out_iters) a.out_iters[s] = k;
+            if (a.out_relres) a.out_relres[s] = relres;
+        }
+    }
+}
+
 // ---------------------------------------------------- cluster kernel ----
 // One thread-block cluster per system (kClusterCTAs blocks): each block owns a
 // contiguous run of rows and keeps its rows' matrix entries, x, r, M^-1, q and
@@ -1363,6 +1508,41 @@ sla_status cg_tile_deps(Csr *h, cudaStream_t s) {
     return SLA_OK;
 }
 
+static const void *pick_segment(sla_dtype dt, int lanes) {
+    const void *f = nullptr;
+    with_lanes(lanes, [&](auto L) -> sla_status {
+        constexpr int LN = decltype(L)::value;
+        f = dt == SLA_F64 ? reinterpret_cast<const void *>(&cg_segment_kernel<double, LN>)
+                          : reinterpret_cast<const void *>(&cg_segment_kernel<float, LN>);
+        return SLA_OK;
+    });
+    return f;
+}
+
+// Segment solver layout of a list handle: shared memory for the vectors of
+// the largest item if it fits (else as many rows as fit; larger items use the
+// workspace vectors), and as many resident blocks as that allows.
+sla_status cg_configure_list(Csr *h) {
+    const size_t ts = dtype_size(h->dtype);
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+    const void *f = pick_segment(h->dtype, h->lanes);
+    sla_status st = smem_ceiling(f, h->device);
+    if (st != SLA_OK) return st;
+    const int64_t cap_rows = (int64_t)(optin - 8192) / (int64_t)(5 * ts);
+    h->seg_smem_rows = (int32_t)std::min<int64_t>(h->seg_max, cap_rows);
+    h->seg_smem = 5 * (size_t)h->seg_smem_rows * ts;
+    int per_sm = 0;
+    SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kCgThreads, h->seg_smem));
+    if (per_sm < 1) {
+        set_error("sla_csr_list_create: the segment solver cannot be resident");
+        return SLA_ERR_CUDA;
+    }
+    const int64_t blocks = (int64_t)per_sm * h->num_sms;
+    h->seg_grid = (int32_t)std::max<int64_t>(1, std::min<int64_t>(h->n_items, blocks));
+    return SLA_OK;
+}
+
 static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
     const size_t ts = dtype_size(h->dtype);
     const size_t B = h->batch, n = h->n_rows, ntot = B * (size_t)h->ntiles;
@@ -1421,6 +1601,21 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
         a.dep_lo = h->dep_lo;
         a.dep_hi = h->dep_hi;
         a.pflag = c.take<unsigned>((size_t)h->ntiles);
+    }
+    if (h->n_items > 0) {
+        SLA_REQUIRE(o->strategy == SLA_STRATEGY_AUTO || o->strategy == SLA_STRATEGY_BLOCK,
+                    "sla_cg: a list of systems is solved one item a block (AUTO or BLOCK strategy)");
+        SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
+        const int32_t *seg = h->seg, *order = h->seg_order;
+        const int n_items = h->n_items, smem_rows = h->seg_smem_rows;
+        unsigned *work = a.sync + 4;
+        return with_lanes(h->lanes, [&](auto L) -> sla_status {
+            constexpr int LN = decltype(L)::value;
+            cg_segment_kernel<T, LN><<<h->seg_grid, kCgThreads, h->seg_smem, s>>>(
+                a, seg, order, n_items, smem_rows, work);
+            SLA_CHECK_LAUNCH();
+            return SLA_OK;
+        });
     }
     bool use_grid = true, use_cluster = false;
     if (o->strategy == SLA_STRATEGY_BLOCK) {
@@ -1504,8 +1699,9 @@ static sla_status cg_entry(Csr *h, const void *vals, const void *rhs, void *x,
     SLA_REQUIRE(h->n_rows == h->n_cols, "sla_cg: matrix must be square (%d x %d)", h->n_rows, h->n_cols);
     cudaStream_t s = as_stream(stream);
     if (h->n_rows == 0) {
-        info_fill_kernel<<<(h->batch + 255) / 256, 256, 0, s>>>(h->batch, info.iters, info.relres,
-                                                                 info.status);
+        const int count = h->n_items > 0 ? h->n_items : h->batch;
+        info_fill_kernel<<<(count + 255) / 256, 256, 0, s>>>(count, info.iters, info.relres,
+                                                             info.status);
         SLA_CHECK_LAUNCH();
         return SLA_OK;
     }

@@ -105,6 +105,15 @@ struct Csr {
     size_t cluster_smem = 0;           // its dynamic shared memory
     int32_t *dep_lo = nullptr, *dep_hi = nullptr;  // owned [ntiles]: tiles a tile's gathers reach
     int32_t block_grid = 0;            // blocks of the block solver (each loops over systems)
+    // A list of independent systems (block-diagonal pattern; see sla_csr_list_create):
+    // item s owns rows and columns [seg[s], seg[s+1]).
+    int32_t n_items = 0;
+    int32_t *seg = nullptr;            // owned [n_items + 1]
+    int32_t *seg_order = nullptr;      // owned [n_items]: items by decreasing size
+    int32_t seg_max = 0;               // rows of the largest item
+    int32_t seg_smem_rows = 0;         // items up to this size keep their vectors in shared memory
+    int32_t seg_grid = 0;              // blocks of the segment solver
+    size_t seg_smem = 0;               // its dynamic shared memory per block
     // Sliced layout of the pattern for the solver's short-row SpMV (see sla_sell.cu):
     // slices of kSellRows consecutive rows, entry k of the slice's rows stored
     // together (padded to the slice's longest row).

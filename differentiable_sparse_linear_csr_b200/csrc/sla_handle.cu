@@ -5,6 +5,8 @@
 #include <climits>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
+#include <vector>
 
 #include "sla_common.cuh"
 
@@ -157,6 +159,31 @@ sla_status ensure_transpose(Csr *h, cudaStream_t s) {
 
 // Persistent-grid and block-solver layout for the handle (in sla_cg.cu).
 sla_status cg_configure(Csr *h);
+// Segment-solver layout of a list handle (in sla_cg.cu).
+sla_status cg_configure_list(Csr *h);
+
+// Every entry of a list handle's row lies in its item's diagonal block:
+// row i of item s (seg[s] <= i < seg[s+1]) may only hold columns in the same
+// range.  The first offending entry is reported as code 7.
+__global__ void list_check_kernel(int n_rows, const int32_t *rowptr, const int32_t *colind,
+                                  int n_items, const int32_t *seg, unsigned long long *best) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n_rows) return;
+    int lo = 0, hi = n_items - 1;           // the item s with seg[s] <= i < seg[s+1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seg[mid] <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    const int c0 = seg[lo], c1 = seg[lo + 1];
+    for (int t = rowptr[i]; t < rowptr[i + 1]; ++t) {
+        const int c = colind[t];
+        if (c < c0 || c >= c1) {
+            atomicMin(best, (7ull << 40) | (unsigned long long)t);
+            return;
+        }
+    }
+}
 
 }  // namespace sla
 
@@ -180,11 +207,102 @@ extern "C" sla_status sla_csr_check(int32_t n_rows, int32_t n_cols, int64_t nnz,
                          as_stream(stream));
 }
 
+namespace {
+sla_status create_handle(int32_t n_rows, int32_t n_cols, int64_t nnz, const int32_t *rowptr,
+                         const int32_t *colind, int32_t batch, sla_dtype dtype, uint32_t flags,
+                         void *stream, sla_csr_t *out, bool list);
+}
+
 extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz,
                                      const int32_t *rowptr, const int32_t *colind,
                                      int32_t batch, sla_dtype dtype, uint32_t flags,
                                      void *stream, sla_csr_t *out) {
     clear_error();
+    return create_handle(n_rows, n_cols, nnz, rowptr, colind, batch, dtype, flags, stream, out, false);
+}
+
+extern "C" sla_status sla_csr_list_create(int32_t n_items, const int32_t *item_rows, int32_t n_rows,
+                                          int64_t nnz, const int32_t *rowptr, const int32_t *colind,
+                                          sla_dtype dtype, uint32_t flags, void *stream,
+                                          sla_csr_t *out) {
+    clear_error();
+    SLA_REQUIRE(out != nullptr, "sla_csr_list_create: NULL out");
+    *out = nullptr;
+    SLA_REQUIRE(n_items >= 1, "sla_csr_list_create: n_items must be >= 1 (got %d)", n_items);
+    SLA_REQUIRE(item_rows != nullptr, "sla_csr_list_create: NULL item_rows");
+    SLA_REQUIRE(n_rows >= 0, "sla_csr_list_create: negative size");
+    std::vector<int32_t> seg((size_t)n_items + 1);
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(seg.data(), item_rows, seg.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        set_error("sla_csr_list_create: cannot read item_rows");
+        return SLA_ERR_CUDA;
+    }
+    SLA_REQUIRE(seg[0] == 0 && seg[n_items] == n_rows,
+                "sla_csr_list_create: item_rows must run from 0 to n_rows (%d .. %d, n_rows %d)", seg[0],
+                seg[n_items], n_rows);
+    int32_t seg_max = 0;
+    for (int32_t i = 0; i < n_items; ++i) {
+        SLA_REQUIRE(seg[i + 1] >= seg[i], "sla_csr_list_create: item_rows decreases at item %d", i);
+        seg_max = std::max(seg_max, seg[i + 1] - seg[i]);
+    }
+    sla_csr_t hh = nullptr;
+    sla_status st = create_handle(n_rows, n_rows, nnz, rowptr, colind, 1, dtype, flags, stream, &hh, true);
+    if (st != SLA_OK) return st;
+    Csr *h = reinterpret_cast<Csr *>(hh);
+    auto fail = [&](sla_status e) {
+        sla_csr_destroy(hh);
+        return e;
+    };
+    std::vector<int32_t> order(n_items);
+    for (int32_t i = 0; i < n_items; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int32_t a, int32_t b) { return seg[a + 1] - seg[a] > seg[b + 1] - seg[b]; });
+    unsigned long long *best = nullptr;
+    if (cudaMalloc(&h->seg, seg.size() * sizeof(int32_t)) != cudaSuccess ||
+        cudaMalloc(&h->seg_order, order.size() * sizeof(int32_t)) != cudaSuccess ||
+        cudaMalloc(&best, sizeof(unsigned long long)) != cudaSuccess) {
+        cudaFree(best);
+        set_error("sla_csr_list_create: out of device memory");
+        return fail(SLA_ERR_OOM);
+    }
+    unsigned long long code = ~0ull;
+    if (cudaMemcpyAsync(h->seg, seg.data(), seg.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(h->seg_order, order.data(), order.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        cudaMemsetAsync(best, 0xff, sizeof(unsigned long long), s) != cudaSuccess) {
+        cudaFree(best);
+        set_error("sla_csr_list_create: copy failed");
+        return fail(SLA_ERR_CUDA);
+    }
+    if (n_rows > 0)
+        list_check_kernel<<<(n_rows + 255) / 256, 256, 0, s>>>(n_rows, rowptr, colind, n_items, h->seg, best);
+    const bool ok = cudaGetLastError() == cudaSuccess &&
+                    cudaMemcpyAsync(&code, best, sizeof(code), cudaMemcpyDeviceToHost, s) == cudaSuccess &&
+                    cudaStreamSynchronize(s) == cudaSuccess;
+    cudaFree(best);
+    if (!ok) {
+        set_error("sla_csr_list_create: block check failed");
+        return fail(SLA_ERR_CUDA);
+    }
+    if (code != ~0ull) {
+        set_error("sla_csr_list_create: entry %lld lies outside its item's diagonal block",
+                  (long long)(code & ((1ull << 40) - 1)));
+        return fail(SLA_ERR_INVALID);
+    }
+    h->n_items = n_items;
+    h->seg_max = seg_max;
+    st = cg_configure_list(h);
+    if (st != SLA_OK) return fail(st);
+    *out = hh;
+    return SLA_OK;
+}
+
+namespace {
+sla_status create_handle(int32_t n_rows, int32_t n_cols, int64_t nnz, const int32_t *rowptr,
+                         const int32_t *colind, int32_t batch, sla_dtype dtype, uint32_t flags,
+                         void *stream, sla_csr_t *out, bool list) {
     SLA_REQUIRE(out != nullptr, "sla_csr_create: NULL out");
     *out = nullptr;
     SLA_REQUIRE(n_rows >= 0 && n_cols >= 0, "sla_csr_create: negative size");
@@ -266,7 +384,7 @@ extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz
         st = diag_positions(n_rows, rowptr, colind, h->diagpos, s);
         if (st != SLA_OK) return fail(st);
     }
-    if (n_rows == n_cols) {
+    if (n_rows == n_cols && !list) {
         st = cg_configure(h);
         if (st == SLA_OK) st = cg_tile_deps(h, s);
         if (st != SLA_OK) return fail(st);
@@ -283,6 +401,7 @@ extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz
     *out = reinterpret_cast<sla_csr_t>(h);
     return SLA_OK;
 }
+}  // namespace
 
 extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     Csr *h = reinterpret_cast<Csr *>(hh);
@@ -297,6 +416,8 @@ extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     cudaFree(h->sell_map);
     cudaFree(h->dep_lo);
     cudaFree(h->dep_hi);
+    cudaFree(h->seg);
+    cudaFree(h->seg_order);
     delete h;
     return SLA_OK;
 }
@@ -322,6 +443,9 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->sliced = h->has_sell ? 1 : 0;
     p->block_resident = h->block_mres ? 1 : 0;
     p->cluster_fits = h->cluster_fits ? 1 : 0;
+    p->n_items = h->n_items;
+    p->item_rows_max = h->seg_max;
+    p->item_smem_rows = h->seg_smem_rows;
     return SLA_OK;
 }
 

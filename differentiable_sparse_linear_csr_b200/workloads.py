@@ -277,6 +277,8 @@ class Workload:
     edges: tuple | None = None
     weights: np.ndarray | None = None
     shift: float = 0.0
+    # lists of independent systems only: item s owns rows [item_rows[s], item_rows[s+1])
+    item_rows: np.ndarray | None = None
 
     @property
     def nnz(self) -> int:
@@ -334,6 +336,33 @@ def c4_batched(seed: int = 4, B: int = 1024, N: int = 32) -> Workload:
                     uniform(seed, STREAM_XSTAR, B * n, -1, 1).reshape(B, n),
                     1e-10, 0, f"{B} shared-pattern {N}x{N} diffusion systems + 1e-2 I, PCG to 1e-10",
                     (ei, ej), w, 1e-2)
+
+
+def list_of_grids(seed: int = 6, B: int = 1024, N_lo: int = 16, N_hi: int = 48) -> Workload:
+    """B independent diffusion systems on N_s x N_s grids, N_s uniform in
+    [N_lo, N_hi] (sizes from the points stream), each L_w + 1e-2 I with
+    w ~ U[0.5, 2] per edge, stored block-diagonally; b ~ N(0,1), x* ~ U[-1,1]."""
+    sizes = N_lo + np.floor(uniform01(seed, STREAM_POINTS, np.arange(B, dtype=np.uint64))
+                            * (N_hi - N_lo + 1)).astype(np.int64)
+    rps, cis, vs, rows, ents, woff = [], [], [], [0], [0], 0
+    for N in sizes:
+        ei, ej = grid_edges((int(N), int(N)))
+        w = uniform(seed, STREAM_WEIGHTS, ei.shape[0], 0.5, 2.0, offset=woff)
+        woff += ei.shape[0]
+        rp, ci, v = weighted_laplacian(int(N) * int(N), ei, ej, w, 1e-2)
+        rps.append(rp[:-1].astype(np.int64) + ents[-1])
+        cis.append(ci.astype(np.int64) + rows[-1])
+        vs.append(v)
+        rows.append(rows[-1] + int(N) * int(N))
+        ents.append(ents[-1] + ci.shape[0])
+    rowptr = np.concatenate(rps + [np.array([ents[-1]])]).astype(np.int32)
+    colind = np.concatenate(cis).astype(np.int32)
+    n = rows[-1]
+    return Workload(f"list_{B}_grids_{N_lo}to{N_hi}", n, rowptr, colind, np.concatenate(vs)[None, :],
+                    _as_batch(normal(seed, STREAM_B, n)), _as_batch(uniform(seed, STREAM_XSTAR, n, -1, 1)),
+                    1e-10, 0, f"list of {B} diffusion systems on N x N grids, N uniform in "
+                              f"[{N_lo}, {N_hi}], + 1e-2 I, PCG to 1e-10",
+                    item_rows=np.array(rows, dtype=np.int32))
 
 
 def c5_knn(seed: int = 5, npts: int = 8_000_000, k: int = 8, order: str = "generated") -> Workload:

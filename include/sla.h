@@ -136,6 +136,10 @@ typedef struct {
     int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
                                  system in shared memory as well as its vectors */
     int32_t cluster_fits;     /* 1 if one system fits the cluster solver */
+    int32_t n_items;          /* list handles: number of items (0 otherwise) */
+    int32_t item_rows_max;    /* list handles: rows of the largest item */
+    int32_t item_smem_rows;   /* list handles: items up to this size keep their vectors in
+                                 shared memory (larger ones use the workspace) */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */
@@ -298,6 +302,30 @@ sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t *rowptr,
                                 const int32_t *colind, int32_t batch, sla_dtype dtype,
                                 const void *vals, const void *b, void *x,
                                 const sla_cg_opts *opts, sla_cg_info info, void *stream);
+
+/*
+ * A list of independent square systems, each with its own pattern (the
+ * SparseTensorList of torch-sla, technical summary, "Methodology" 1: a batch
+ * whose items have different patterns).  The caller stores the items as one
+ * block-diagonal CSR: item s owns rows and columns [item_rows[s],
+ * item_rows[s+1]) (device int32 [n_items + 1], read during the call only;
+ * item_rows[0] = 0, non-decreasing, item_rows[n_items] = n_rows) and its
+ * entries keep global column indices.  rowptr/colind are borrowed as for
+ * sla_csr_create; flags as there (VALIDATE checks the CSR rules; the block
+ * structure is always checked: an entry outside its item's block is
+ * SLA_ERR_INVALID).  Synchronises the host.
+ *
+ * The handle has batch 1: values [nnz], vectors [n_rows].  sla_spmv and
+ * sla_grad_values act on the whole block-diagonal matrix, which is each item's
+ * own product.  sla_cg_solve / sla_cg_adjoint solve every item independently
+ * (its own alpha, beta, stop test relative to its own ||b||) and write
+ * sla_cg_info per item ([n_items]); strategy AUTO or BLOCK (each item runs in
+ * one thread block, largest items first; items too large for shared memory
+ * use the workspace vectors).
+ */
+sla_status sla_csr_list_create(int32_t n_items, const int32_t *item_rows, int32_t n_rows,
+                               int64_t nnz, const int32_t *rowptr, const int32_t *colind,
+                               sla_dtype dtype, uint32_t flags, void *stream, sla_csr_t *out);
 
 /*
  * Edge-weighted graph Laplacian on a handle's pattern: the map from edge

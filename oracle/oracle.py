@@ -360,3 +360,33 @@ def newton_adjoint(rowptr, colind, jac_values, gu, *, cg_rtol=1e-13):
     vector-Jacobian product with -lambda."""
     lam, _ = cg_adjoint(rowptr, colind, jac_values, gu, rtol=cg_rtol)
     return lam
+
+
+def _items(item_rows, rowptr, colind):
+    """Each item's own CSR (local row and column numbers) and its row / entry ranges."""
+    item_rows, rowptr, colind = np.asarray(item_rows), _i32(rowptr), _i32(colind)
+    for s in range(item_rows.shape[0] - 1):
+        o, e = int(item_rows[s]), int(item_rows[s + 1])
+        t0, t1 = int(rowptr[o]), int(rowptr[e])
+        yield o, e, t0, t1, (rowptr[o:e + 1] - t0).astype(np.int32), (colind[t0:t1] - o).astype(np.int32)
+
+
+def pcg_list(item_rows, rowptr, colind, vals, b, *, adjoint=False, **kw):
+    """Independent Jacobi-PCG solves of the items of a block-diagonal CSR
+    (torch-sla's SparseTensorList, technical summary, "Methodology" 1): item s
+    owns rows and columns [item_rows[s], item_rows[s+1]).  Returns the
+    concatenated solution and a SolveInfo with one entry per item."""
+    vals, b = np.asarray(vals), np.asarray(b)
+    x = np.zeros_like(b)
+    iters, status, relres = [], [], []
+    x0 = kw.pop("x0", None)
+    for o, e, t0, t1, rp, ci in _items(item_rows, rowptr, colind):
+        if x0 is not None:
+            kw["x0"] = np.asarray(x0)[o:e]
+        fn = cg_adjoint if adjoint else pcg
+        xs, info = fn(rp, ci, vals[t0:t1], b[o:e], **kw)
+        x[o:e] = xs
+        iters.append(int(np.atleast_1d(info.iters)[0]))
+        status.append(int(np.atleast_1d(info.status)[0]))
+        relres.append(float(np.atleast_1d(info.relres)[0]))
+    return x, SolveInfo(np.array(iters), np.array(status), np.array(relres))
