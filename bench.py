@@ -141,8 +141,8 @@ class ClockSampler:
 
 _WORKLOAD = {}
 
-WORKLOADS = ("c2", "c1", "c3", "c4", "c5", "c5rcm")
-CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12}
+WORKLOADS = ("c2", "c1", "c3", "c4", "c5", "c5rcm", "c4list")
+CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12, "c4list": 60}
 
 
 def load_workload(name: str, rank: int = 0):
@@ -162,6 +162,8 @@ def load_workload(name: str, rank: int = 0):
             w = W.c5_knn(seed=5 + 10 * rank)
         elif name == "c5rcm":
             w = W.c5_knn(seed=5 + 10 * rank, order="rcm")
+        elif name == "c4list":
+            w = W.list_of_grids(seed=6 + 10 * rank)
         else:
             raise ValueError(name)
         _WORKLOAD[key] = w
@@ -178,6 +180,18 @@ def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2", edges: bool =
     npdt = np.float64 if dtype_name == "f64" else np.float32
     v, b, xs = w.values[0].astype(npdt), w.b[0].astype(npdt), w.xstar[0].astype(npdt)
     O.build()
+    if w.item_rows is not None:
+        # a list: its first 32 items, each k forward + k adjoint iterations
+        ir = w.item_rows[:33]
+        e = int(w.rowptr[ir[-1]])
+        rp, ci = w.rowptr[:ir[-1] + 1], w.colind[:e]
+        t0 = time.perf_counter()
+        x, _ = O.pcg_list(ir, rp, ci, v[:e], b[:ir[-1]], fixed_iters=k_iters)
+        lam, _ = O.pcg_list(ir, rp, ci, v[:e], (x - xs[:ir[-1]]).astype(npdt), adjoint=True,
+                            fixed_iters=k_iters)
+        O.grad_values(rp, ci, lam, x)
+        dt = time.perf_counter() - t0
+        return 2 * 32 * k_iters / dt, dt
     t0 = time.perf_counter()
     if edges:
         v = O.laplacian_assemble(w.rowptr, w.colind, w.edges[0], w.edges[1],
@@ -216,8 +230,8 @@ def run_reference(args):
         oracle_sample(args.dtype, k, args.workload, args.edges)
     total_it, total_t = 0, 0.0
     for _ in range(args.steps):
-        _, dt = oracle_sample(args.dtype, k, args.workload, args.edges)
-        total_it += 2 * k
+        rate, dt = oracle_sample(args.dtype, k, args.workload, args.edges)
+        total_it += rate * dt                     # iterations of the sample (items x 2k for a list)
         total_t += dt
     v = total_it / total_t
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
@@ -226,7 +240,8 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
             "config": workload_config(args),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": f"each step: {k} forward + {k} adjoint PCG iterations + "
+                             "sample": f"each step: {k} forward + {k} adjoint PCG iterations "
+                                       f"{'of each of the first 32 items ' if args.workload == 'c4list' else ''}+ "
                                        f"{'edge-weight' if args.edges else 'value'} gradient of "
                                        f"system 0 of workload {args.workload}"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -247,6 +262,7 @@ def workload_config(args, w=None):
         what = f"{w.description}: {mode} Jacobi-PCG iterations + sparse value gradient"
     return {"workload": what, "edges": bool(args.edges),
             "name": args.workload, "n": int(w.n), "nnz": int(w.nnz), "batch": int(w.batch),
+            **({"items": int(len(w.item_rows) - 1)} if w.item_rows is not None else {}),
             "value_dtype": args.dtype, "l2": "flushed between steps (write of a 256 MiB buffer)",
             "parallelism": f"replicas x{world}"}
 
@@ -297,8 +313,12 @@ def main():
     w = load_workload(args.workload, rank)
     n, nnz, B = w.n, w.nnz, w.batch
     fixed = args.iters if args.iters > 0 else w.fixed_iters
-    A = sla.CSR(torch.from_numpy(w.rowptr).to(dev), torch.from_numpy(w.colind).to(dev),
-                batch=B, dtype=dt, symmetric=True)
+    if w.item_rows is not None:
+        A = sla.CSRList(torch.from_numpy(w.item_rows).to(dev), torch.from_numpy(w.rowptr).to(dev),
+                        torch.from_numpy(w.colind).to(dev), dtype=dt, symmetric=True)
+    else:
+        A = sla.CSR(torch.from_numpy(w.rowptr).to(dev), torch.from_numpy(w.colind).to(dev),
+                    batch=B, dtype=dt, symmetric=True)
     vals = torch.from_numpy(w.values).to(dev, dt).contiguous()
     b = torch.from_numpy(w.b).to(dev, dt).contiguous()
     xs = torch.from_numpy(w.xstar).to(dev, dt).contiguous()
@@ -306,8 +326,8 @@ def main():
     g = torch.empty(B, n, dtype=dt, device=dev)
     lam = torch.empty(B, n, dtype=dt, device=dev)
     G = torch.empty(B, nnz, dtype=dt, device=dev)
-    finfo = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
-    ainfo = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    finfo = [torch.empty(A.n_info, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    ainfo = [torch.empty(A.n_info, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
     ws = torch.empty(L.sla_workspace_bytes(A.handle, L.SLA_OP_ADJOINT), dtype=torch.uint8, device=dev)
     opts = L.make_opts(rtol=w.rtol, fixed_iters=fixed, strategy=args.strategy)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -419,7 +439,8 @@ def main():
 
     if rank == 0:
         peak, peak_kind = measured_hbm_peak()
-        it_bytes = per_iteration_bytes(n, nnz, vbytes)
+        # a list: the mean item's bytes per item-iteration
+        it_bytes = per_iteration_bytes(n // A.n_info, nnz // A.n_info, vbytes)
         cg_ms = statistics.mean(fwd_ms) + statistics.mean(adj_ms)
         achieved = (fwd_it + adj_it) * it_bytes / (cg_ms / 1000.0) / 1e9
         props = A.props
@@ -432,7 +453,11 @@ def main():
         if args.edges:
             # assembly; the edge gradient (per edge) and the shift gradient (tile sums, finish)
             launches_per_step += 1 + 2
-        if uses_cluster:
+        if w.item_rows is not None:
+            uses_cluster = uses_grid = False
+            launches_per_step = 3
+            variant = "one block per item, largest items first"
+        elif uses_cluster:
             variant = "thread-block cluster per system, DSMEM"
         elif not uses_grid:
             variant = ("block-per-system, whole system in shared memory" if props.block_resident
