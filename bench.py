@@ -141,8 +141,9 @@ class ClockSampler:
 
 _WORKLOAD = {}
 
-WORKLOADS = ("c2", "c1", "c3", "c4", "c5", "c5rcm", "c4list")
-CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12, "c4list": 60}
+WORKLOADS = ("c2", "c1", "c3", "c4", "c5", "c5rcm", "c4list", "c3b4")
+CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12, "c4list": 60,
+             "c3b4": 100}
 
 
 def load_workload(name: str, rank: int = 0):
@@ -164,6 +165,8 @@ def load_workload(name: str, rank: int = 0):
             w = W.c5_knn(seed=5 + 10 * rank, order="rcm")
         elif name == "c4list":
             w = W.list_of_grids(seed=6 + 10 * rank)
+        elif name == "c3b4":
+            w = W.c3_batched(seed=3 + 10 * rank, B=4)
         else:
             raise ValueError(name)
         _WORKLOAD[key] = w
@@ -286,8 +289,8 @@ def main():
                     help="edge-weighted workloads (c3, c4, c5, c5rcm): assemble the values from "
                          "the edge weights and take the gradient back to them")
     args = ap.parse_args()
-    if args.edges and args.workload not in ("c3", "c4", "c5", "c5rcm"):
-        ap.error("--edges needs an edge-weighted workload (c3, c4, c5, c5rcm)")
+    if args.edges and args.workload not in ("c3", "c4", "c5", "c5rcm", "c3b4"):
+        ap.error("--edges needs an edge-weighted workload (c3, c4, c5, c5rcm, c3b4)")
     if args.impl == "reference":
         return run_reference(args)
 
@@ -439,8 +442,11 @@ def main():
 
     if rank == 0:
         peak, peak_kind = measured_hbm_peak()
-        # a list: the mean item's bytes per item-iteration
-        it_bytes = per_iteration_bytes(n // A.n_info, nnz // A.n_info, vbytes)
+        # per system-iteration (a list: the mean item's bytes per item-iteration)
+        if w.item_rows is not None:
+            it_bytes = per_iteration_bytes(n // A.n_info, nnz // A.n_info, vbytes)
+        else:
+            it_bytes = per_iteration_bytes(n, nnz, vbytes)
         cg_ms = statistics.mean(fwd_ms) + statistics.mean(adj_ms)
         achieved = (fwd_it + adj_it) * it_bytes / (cg_ms / 1000.0) / 1e9
         props = A.props
@@ -462,6 +468,9 @@ def main():
         elif not uses_grid:
             variant = ("block-per-system, whole system in shared memory" if props.block_resident
                        else "block-per-system, vectors in shared memory")
+        elif props.interleaved:
+            variant = "persistent grid, batch interleaved [entry][system], vectors in HBM"
+            launches_per_step = 2 * 4 + 1          # layouts in and out, values, solver
         elif props.grid_onchip == 2:
             variant = "persistent grid, x, r, M^-1 on chip, two barriers an iteration"
         elif props.grid_onchip:

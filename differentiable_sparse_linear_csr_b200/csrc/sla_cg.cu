@@ -119,6 +119,19 @@ __device__ __forceinline__ void system_sums(const double *const (&arr)[NV], int 
     block_sums<NT, NV>(out, red);
 }
 
+// system_sums for an array of partial pointers built at run time.
+template <int NT, int NV>
+__device__ __forceinline__ void system_sums_dyn(const double *const *arr, int ntiles, double (&out)[NV],
+                                                double *red) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        double acc = 0.0;
+        for (int j = threadIdx.x; j < ntiles; j += NT) acc += __ldcg(arr[k] + j);
+        out[k] = acc;
+    }
+    block_sums<NT, NV>(out, red);
+}
+
 // Device-wide barrier on a monotonically increasing arrival counter: the k-th
 // barrier of the launch completes when the counter reaches k * gridDim.x, a
 // target every block knows, so arrival is a single fire-and-forget add and the
@@ -835,6 +848,319 @@ cg_block_kernel(CgArgs<T> a) {
     }
 }
 
+// ------------------------------------------- interleaved batch kernel ----
+// The persistent solver for a batch of BW systems sharing a pattern, with the
+// values laid out [entry][system] (the sliced layout's slots, BW values each)
+// and every vector [row][system]: one column-index load and one gather address
+// serve all BW systems, and BW values move in one vector load.  Rows are
+// split into tiles shared by the BW systems, at most one per block.  Each
+// system keeps its own scalars, stop test and iteration count; every block
+// takes the same per-system decisions from the tile partials, and a system
+// that has stopped is left untouched until all have.  The phases and the
+// arithmetic per system are those of cg_grid_kernel.
+template <typename T, int BW>
+struct VecLoad {
+    // BW consecutive values starting at a multiple of BW elements
+    static __device__ __forceinline__ void ld(const T *p, T (&v)[BW]) {
+        constexpr int bytes = BW * (int)sizeof(T);
+        if constexpr (bytes % 16 == 0) {
+#pragma unroll
+            for (int c = 0; c < bytes / 16; ++c) {
+                const float4 u = *reinterpret_cast<const float4 *>(reinterpret_cast<const char *>(p) + 16 * c);
+                memcpy(reinterpret_cast<char *>(v) + 16 * c, &u, 16);
+            }
+        } else if constexpr (bytes == 8) {
+            const float2 u = *reinterpret_cast<const float2 *>(p);
+            memcpy(v, &u, 8);
+        } else {
+#pragma unroll
+            for (int s = 0; s < BW; ++s) v[s] = p[s];
+        }
+    }
+    static __device__ __forceinline__ void st(T *p, const T (&v)[BW]) {
+#pragma unroll
+        for (int s = 0; s < BW; ++s) p[s] = v[s];
+    }
+};
+
+template <typename T, int BW>
+__device__ __forceinline__ void il_row(const int32_t *__restrict__ sptr, const int32_t *__restrict__ cols,
+                                       const T *__restrict__ sv, const T *v, int i, T (&q)[BW]) {
+    const int sl = i / kSellRows;
+    const int b0 = __ldg(sptr + sl);
+    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
+    const int base = b0 + i % kSellRows;
+#pragma unroll
+    for (int s = 0; s < BW; ++s) q[s] = T(0);
+    for (int k = 0; k < w; ++k) {
+        const int t = base + k * kSellRows;
+        const int c = sell_load<true>(cols + t);
+        T av[BW], pv[BW];
+        VecLoad<T, BW>::ld(sv + (int64_t)t * BW, av);
+        VecLoad<T, BW>::ld(v + (int64_t)c * BW, pv);
+#pragma unroll
+        for (int s = 0; s < BW; ++s) q[s] += av[s] * pv[s];
+    }
+}
+
+template <typename T, int BW>
+__global__ void __launch_bounds__(kCgThreads, 2)
+cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, int ntiles) {
+    constexpr int NT = kCgThreads;
+    __shared__ double red[4 * BW * 33];
+    __shared__ double s_rho[BW], s_nb[BW], s_rr[BW], s_alpha[BW];
+    __shared__ int s_state[BW], s_iters[BW];
+    __shared__ int flag;
+    const int tid = threadIdx.x;
+    const int n = a.n;
+    const int tile = blockIdx.x;
+    const bool has_tile = tile < ntiles;
+    const int r0 = tile * tile_rows, r1 = has_tile ? min(n, r0 + tile_rows) : r0;
+    // partial of quantity qn for system s: part[(qn * BW + s) * ntiles + tile]
+    auto P = [&](int qn, int s) { return part + (int64_t)(qn * BW + s) * ntiles; };
+    const T *sv = a.sell_vals;
+    T *r = a.r, *p = a.p, *q = a.q, *d = a.d;
+    unsigned target = 0;
+    auto give_up_il = [&]() {
+        if (tid == 0)
+            for (int s = 0; s < BW; ++s)
+                if (s_state[s] == kActive && a.out_status) a.out_status[s] = SLA_TIMED_OUT;
+    };
+    if (tid < BW) s_state[tid] = kActive;
+
+    // ---- init: r = b - A x0 (or b), M^-1, p = z; partials of b.b, r.z, r.r, bad diagonals
+    {
+        double acc[4 * BW];
+#pragma unroll
+        for (int j = 0; j < 4 * BW; ++j) acc[j] = 0.0;
+        for (int i = r0 + tid; i < r1; i += NT) {
+            T qx[BW];
+            if (a.x0_given) il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, xi, i, qx);
+            const int dp = a.precond ? __ldg(a.diagpos + i) : -1;
+#pragma unroll
+            for (int s = 0; s < BW; ++s) {
+                const int64_t o = (int64_t)i * BW + s;
+                const T b_ = bi[o];
+                const T ri = a.x0_given ? b_ - qx[s] : b_;
+                T di = T(1);
+                if (a.precond) {
+                    const T dv = dp >= 0 ? __ldg(a.vals + (int64_t)s * a.nnz + dp) : T(0);
+                    if (!(dv > T(0))) acc[3 * BW + s] += 1.0;
+                    di = T(1) / dv;
+                }
+                const T zi = di * ri;
+                if (!a.x0_given) xi[o] = T(0);
+                r[o] = ri;
+                d[o] = di;
+                p[o] = zi;
+                acc[s] += (double)b_ * (double)b_;
+                acc[BW + s] += (double)ri * (double)zi;
+                acc[2 * BW + s] += (double)ri * (double)ri;
+            }
+        }
+        block_sums<NT, 4 * BW>(acc, red);
+        if (tid == 0 && has_tile)
+            for (int j = 0; j < 4 * BW; ++j) P(j / BW, j % BW)[tile] = acc[j];
+    }
+    if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up_il(); return; }
+    {
+        const double *arr[4 * BW];
+        for (int j = 0; j < 4 * BW; ++j) arr[j] = P(j / BW, j % BW);
+        double sum[4 * BW];
+        system_sums_dyn<NT, 4 * BW>(arr, ntiles, sum, red);
+        if (tid == 0) {
+            for (int s = 0; s < BW; ++s) {
+                const double nb = sqrt(sum[s]), rho0 = sum[BW + s], rr = sum[2 * BW + s];
+                const double tol = fmax(a.rtol * nb, a.atol);
+                int st = kActive;
+                double relres = 0.0;
+                if (nb == 0.0) st = SLA_CONVERGED;
+                else if (!isfinite(nb)) st = SLA_NONFINITE;
+                else if (a.precond && sum[3 * BW + s] > 0.0) { st = SLA_BREAKDOWN; relres = sqrt(rr) / nb; }
+                else if (!a.fixed && sqrt(rr) <= tol) { st = SLA_CONVERGED; relres = sqrt(rr) / nb; }
+                else if (rr == 0.0) st = SLA_CONVERGED;
+                s_state[s] = st;
+                s_rho[s] = rho0;
+                s_nb[s] = nb;
+                s_rr[s] = rr;
+                s_iters[s] = 0;
+                if (st != kActive && blockIdx.x == 0) finalize(a, s, st, 0, relres, false);
+            }
+        }
+        __syncthreads();
+        // systems with b = 0 report x = 0
+        for (int s = 0; s < BW; ++s)
+            if (s_nb[s] == 0.0)
+                for (int i = r0 + tid; i < r1; i += NT) xi[(int64_t)i * BW + s] = T(0);
+    }
+    auto any_active = [&]() {
+        bool m = false;
+        for (int s = 0; s < BW; ++s) m |= s_state[s] == kActive;
+        return m;
+    };
+    while (any_active()) {
+        bool act[BW];
+#pragma unroll
+        for (int s = 0; s < BW; ++s) act[s] = s_state[s] == kActive;
+        // ---- phase A: q = A p for all systems, partials of p.q
+        {
+            double acc[BW];
+#pragma unroll
+            for (int s = 0; s < BW; ++s) acc[s] = 0.0;
+            for (int i = r0 + tid; i < r1; i += NT) {
+                T qv[BW], pv[BW];
+                il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, p, i, qv);
+                VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
+                VecLoad<T, BW>::st(q + (int64_t)i * BW, qv);
+#pragma unroll
+                for (int s = 0; s < BW; ++s) acc[s] += (double)pv[s] * (double)qv[s];
+            }
+            block_sums<NT, BW>(acc, red);
+            if (tid == 0 && has_tile)
+                for (int s = 0; s < BW; ++s) P(0, s)[tile] = acc[s];
+        }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up_il(); return; }
+        // ---- phase B: alpha per system; r -= alpha q; partials of r.z and r.r
+        {
+            const double *arr[BW];
+            for (int s = 0; s < BW; ++s) arr[s] = P(0, s);
+            double sg[BW];
+            system_sums_dyn<NT, BW>(arr, ntiles, sg, red);
+            if (tid == 0) {
+                for (int s = 0; s < BW; ++s) {
+                    if (!act[s]) continue;
+                    const double sigma = sg[s];
+                    if (!isfinite(sigma) || !(sigma > 0.0)) {
+                        const int st = isfinite(sigma) ? SLA_BREAKDOWN : SLA_NONFINITE;
+                        s_state[s] = st;
+                        if (blockIdx.x == 0) finalize(a, s, st, s_iters[s], sqrt(s_rr[s]) / s_nb[s], false);
+                    } else {
+                        s_alpha[s] = s_rho[s] / sigma;
+                        s_iters[s] += 1;
+                    }
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int s = 0; s < BW; ++s) act[s] = s_state[s] == kActive;
+            T al[BW];
+#pragma unroll
+            for (int s = 0; s < BW; ++s) al[s] = (T)s_alpha[s];
+            double acc[2 * BW];
+#pragma unroll
+            for (int j = 0; j < 2 * BW; ++j) acc[j] = 0.0;
+            for (int i = r0 + tid; i < r1; i += NT) {
+                T rv[BW], qv[BW], dv[BW];
+                VecLoad<T, BW>::ld(r + (int64_t)i * BW, rv);
+                VecLoad<T, BW>::ld(q + (int64_t)i * BW, qv);
+                VecLoad<T, BW>::ld(d + (int64_t)i * BW, dv);
+#pragma unroll
+                for (int s = 0; s < BW; ++s) {
+                    if (!act[s]) continue;
+                    const T ri = rv[s] - al[s] * qv[s];
+                    rv[s] = ri;
+                    const T zi = dv[s] * ri;
+                    acc[s] += (double)ri * (double)zi;
+                    acc[BW + s] += (double)ri * (double)ri;
+                }
+                VecLoad<T, BW>::st(r + (int64_t)i * BW, rv);
+            }
+            block_sums<NT, 2 * BW>(acc, red);
+            if (tid == 0 && has_tile)
+                for (int j = 0; j < 2 * BW; ++j) P(1 + j / BW, j % BW)[tile] = acc[j];
+        }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up_il(); return; }
+        // ---- phase C: stop tests; x += alpha p; beta; p = z + beta p
+        {
+            const double *arr[2 * BW];
+            for (int j = 0; j < 2 * BW; ++j) arr[j] = P(1 + j / BW, j % BW);
+            double sum[2 * BW];
+            system_sums_dyn<NT, 2 * BW>(arr, ntiles, sum, red);
+            __shared__ int s_go[BW];
+            __shared__ double s_beta[BW];
+            if (tid == 0) {
+                for (int s = 0; s < BW; ++s) {
+                    s_go[s] = 0;
+                    if (!act[s]) continue;
+                    const double rho_new = sum[s], rr = sum[BW + s];
+                    const double nb = s_nb[s];
+                    const double tol = fmax(a.rtol * nb, a.atol);
+                    const int k = s_iters[s];
+                    int st = kActive;
+                    if (!isfinite(rr)) st = SLA_NONFINITE;
+                    else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
+                    else if (rr == 0.0) st = SLA_CONVERGED;
+                    else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
+                    s_beta[s] = rho_new / s_rho[s];
+                    s_rr[s] = rr;
+                    if (st == kActive) {
+                        s_go[s] = 1;
+                        s_rho[s] = rho_new;
+                    } else {
+                        s_state[s] = st;
+                        if (blockIdx.x == 0) finalize(a, s, st, k, sqrt(rr) / nb, false);
+                    }
+                }
+            }
+            __syncthreads();
+            T al[BW], bt[BW];
+            bool go[BW];
+#pragma unroll
+            for (int s = 0; s < BW; ++s) {
+                al[s] = (T)s_alpha[s];
+                bt[s] = (T)s_beta[s];
+                go[s] = s_go[s] != 0;
+            }
+            for (int i = r0 + tid; i < r1; i += NT) {
+                T xv[BW], pv[BW], rv[BW], dv[BW];
+                VecLoad<T, BW>::ld(xi + (int64_t)i * BW, xv);
+                VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
+                VecLoad<T, BW>::ld(r + (int64_t)i * BW, rv);
+                VecLoad<T, BW>::ld(d + (int64_t)i * BW, dv);
+#pragma unroll
+                for (int s = 0; s < BW; ++s) {
+                    if (!act[s]) continue;
+                    const T pi = pv[s];
+                    xv[s] = xv[s] + al[s] * pi;
+                    if (go[s]) pv[s] = dv[s] * rv[s] + bt[s] * pi;
+                }
+                VecLoad<T, BW>::st(xi + (int64_t)i * BW, xv);
+                VecLoad<T, BW>::st(p + (int64_t)i * BW, pv);
+            }
+        }
+        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up_il(); return; }
+    }
+}
+
+// Batch-major [B][n] <-> interleaved [n][B].
+template <typename T>
+__global__ void interleave_kernel(int64_t n, int B, const T *__restrict__ in, T *__restrict__ out) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n * B) return;
+    const int64_t i = g / B;
+    const int s = (int)(g % B);
+    out[g] = in[(int64_t)s * n + i];
+}
+template <typename T>
+__global__ void deinterleave_kernel(int64_t n, int B, const T *__restrict__ in, T *__restrict__ out) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n * B) return;
+    const int s = (int)(g / n);
+    const int64_t i = g % n;
+    out[g] = in[i * B + s];
+}
+// The sliced layout's values, slot-major: out[slot * B + s] = vals[s][map[slot]].
+template <typename T>
+__global__ void sell_values_il_kernel(int64_t sell_nnz, int64_t nnz, int B, const int32_t *__restrict__ map,
+                                      const T *__restrict__ vals, T *__restrict__ out) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= sell_nnz * B) return;
+    const int64_t slot = g / B;
+    const int s = (int)(g % B);
+    const int t = map[slot];
+    out[g] = t >= 0 ? vals[(int64_t)s * nnz + t] : T(0);
+}
+
 // ---------------------------------------------------- segment kernel ----
 // A list of independent systems with their own patterns, stored as one
 // block-diagonal CSR whose item s owns rows (and columns) [seg[s], seg[s+1]).
@@ -1292,6 +1618,14 @@ static const void *pick_grid2(sla_dtype dt, int rpt) {
     return rpt <= 8 ? grid2_fn<float, 8>() : grid2_fn<float, 16>();
 }
 
+static const void *pick_il(sla_dtype dt, int B) {
+    if (dt == SLA_F64)
+        return B == 2 ? reinterpret_cast<const void *>(&cg_grid_il_kernel<double, 2>)
+                      : reinterpret_cast<const void *>(&cg_grid_il_kernel<double, 4>);
+    return B == 2 ? reinterpret_cast<const void *>(&cg_grid_il_kernel<float, 2>)
+                  : reinterpret_cast<const void *>(&cg_grid_il_kernel<float, 4>);
+}
+
 static const void *pick_grid(const Csr *h, bool sell) {
     if (h->onchip) return pick_onchip(h->dtype, h->onchip_rpt, sell);
     if (sell) return h->dtype == SLA_F64 ? grid_sell_fn<double>() : grid_sell_fn<float>();
@@ -1410,6 +1744,16 @@ sla_status cg_configure(Csr *h) {
         h->grid_threads = kCgThreads;
         h->grid_smem = 0;
         layout(h, h->grid_blocks, &h->tile_rows, &h->ntiles);
+        // batches of 2 or 4 systems: the interleaved solver (values [entry][system])
+        const char *ie = getenv("SLA_INTERLEAVE");
+        h->il_blocks = 0;
+        if ((h->batch == 2 || h->batch == 4) && n > 0 && !(ie && ie[0] == '0')) {
+            const void *f = pick_il(h->dtype, h->batch);
+            int per_il = 0;
+            SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_il, f, kCgThreads, 0));
+            per_il = std::min(per_il, 2);
+            if (per_il >= 1) h->il_blocks = per_il * h->num_sms;
+        }
     }
     // Cluster solver: rows split over kClusterCTAs blocks on 32-row boundaries,
     // each block's matrix slice, vectors and p in its shared memory.
@@ -1550,6 +1894,8 @@ static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
     b += 4 * align_up(B * n * ts);
     if (h->has_sell) b += align_up(B * (size_t)h->sell_nnz * ts);
     b += align_up((size_t)h->ntiles * 4);   // p-ready flags
+    if (h->il_blocks > 0)                   // interleaved x and b, tile partials
+        b += 2 * align_up(B * n * ts) + align_up(4 * B * (size_t)h->il_blocks * 8);
     if (adjoint && !(h->flags & SLA_FLAG_SYMMETRIC)) b += align_up(B * (size_t)h->nnz * ts);
     return b;
 }
@@ -1655,6 +2001,34 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
         }
         // short rows on the forward pattern: the sliced layout, values laid out now
         const bool sell = h->has_sell && pattern_is_forward;
+        if (sell && h->il_blocks > 0 && !h->onchip && (a.B == 2 || a.B == 4)) {
+            // interleaved batch: values [slot][system], vectors [row][system]
+            const int64_t n64 = a.n;
+            T *sv = c.take<T>((size_t)a.B * h->sell_nnz);
+            T *xi = c.take<T>((size_t)a.B * a.n);
+            T *bi = c.take<T>((size_t)a.B * a.n);
+            double *part = c.take<double>(4 * (size_t)a.B * h->il_blocks);
+            const int tile_rows = (int)((n64 + h->il_blocks - 1) / h->il_blocks);
+            const int ntiles = (int)((n64 + tile_rows - 1) / tile_rows);
+            const unsigned gv = (unsigned)((n64 * a.B + 255) / 256);
+            const unsigned gs = (unsigned)((h->sell_nnz * a.B + 255) / 256);
+            sell_values_il_kernel<T><<<gs, 256, 0, s>>>(h->sell_nnz, h->nnz, a.B, h->sell_map, vals, sv);
+            interleave_kernel<T><<<gv, 256, 0, s>>>(n64, a.B, b, bi);
+            if (a.x0_given) interleave_kernel<T><<<gv, 256, 0, s>>>(n64, a.B, x, xi);
+            SLA_CHECK_LAUNCH();
+            a.sell_ptr = h->sell_ptr;
+            a.sell_cols = h->sell_cols;
+            a.sell_vals = sv;
+            a.sell_nnz = h->sell_nnz;
+            SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
+            const T *bic = bi;
+            void *args[] = {&a, &xi, &bic, &part, (void *)&tile_rows, (void *)&ntiles};
+            SLA_CHECK_CUDA(cudaLaunchCooperativeKernel(pick_il(h->dtype, a.B), dim3(h->il_blocks),
+                                                       dim3(kCgThreads), args, 0, s));
+            deinterleave_kernel<T><<<gv, 256, 0, s>>>(n64, a.B, xi, x);
+            SLA_CHECK_LAUNCH();
+            return SLA_OK;
+        }
         if (sell) {
             T *sv = c.take<T>((size_t)a.B * h->sell_nnz);
             sla_status st = sell_values(h, vals, sv, s);

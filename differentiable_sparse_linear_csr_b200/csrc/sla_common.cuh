@@ -105,6 +105,7 @@ struct Csr {
     size_t cluster_smem = 0;           // its dynamic shared memory
     int32_t *dep_lo = nullptr, *dep_hi = nullptr;  // owned [ntiles]: tiles a tile's gathers reach
     int32_t block_grid = 0;            // blocks of the block solver (each loops over systems)
+    int32_t il_blocks = 0;             // batches of 2 or 4 in HBM: interleaved solver grid (0: none)
     // A list of independent systems (block-diagonal pattern; see sla_csr_list_create):
     // item s owns rows and columns [seg[s], seg[s+1]).
     int32_t n_items = 0;

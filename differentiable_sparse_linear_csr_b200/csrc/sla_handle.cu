@@ -446,6 +446,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->n_items = h->n_items;
     p->item_rows_max = h->seg_max;
     p->item_smem_rows = h->seg_smem_rows;
+    p->interleaved = h->il_blocks > 0 && h->has_sell && !h->onchip ? 1 : 0;
     return SLA_OK;
 }
 

@@ -325,6 +325,23 @@ def c3_diffusion3d(seed: int = 3, N: int = 128) -> Workload:
                     (ei, ej), w[None, :], 1e-3)
 
 
+def c3_batched(seed: int = 3, N: int = 128, B: int = 4) -> Workload:
+    """B systems sharing the 3-D 7-point pattern of an N^3 grid, each with its own
+    log-normal weights (w = exp(N(0,1)) per edge, system s drawing indices
+    [s E, (s+1) E) of the weights stream) + 1e-3 I; b, x* ~ U[-1,1] per system."""
+    dims = (N, N, N)
+    n = N ** 3
+    ei, ej = grid_edges(dims)
+    m = ei.shape[0]
+    w = np.exp(normal(seed, STREAM_WEIGHTS, B * m)).reshape(B, m)
+    rp, ci, v = weighted_laplacian(n, ei, ej, w, 1e-3)
+    return Workload(f"c3_batched_{B}x{N}^3", n, rp, ci, v,
+                    uniform(seed, STREAM_B, B * n, -1, 1).reshape(B, n),
+                    uniform(seed, STREAM_XSTAR, B * n, -1, 1).reshape(B, n),
+                    1e-8, 0, f"{B} shared-pattern 3-D 7-point log-normal diffusion systems {N}^3 + 1e-3 I, "
+                             f"PCG to 1e-8", (ei, ej), w, 1e-3)
+
+
 def c4_batched(seed: int = 4, B: int = 1024, N: int = 32) -> Workload:
     n = N * N
     ei, ej = grid_edges((N, N))

@@ -140,6 +140,11 @@ typedef struct {
     int32_t item_rows_max;    /* list handles: rows of the largest item */
     int32_t item_smem_rows;   /* list handles: items up to this size keep their vectors in
                                  shared memory (larger ones use the workspace) */
+    int32_t interleaved;      /* 1 if forward (and symmetric adjoint) grid solves of this
+                                 batch of 2 or 4 systems run the interleaved solver: values
+                                 [entry][system] and vectors [row][system] in the workspace,
+                                 one column index and gather address for all systems.
+                                 SLA_INTERLEAVE=0, read at creation, turns it off */
 } sla_csr_props;
 
 /* Operations for sla_workspace_bytes. */
