@@ -72,17 +72,25 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kernel_key: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+def profile_traffic(kernel_key: str, iters_per_launch: float):
+    """DRAM bytes per launch from a committed ncu summary whose source digest
+    matches the library source: either a per-launch figure, or a per-iteration
+    figure (for kernels whose traffic grows with the iteration count) scaled to
+    this launch's iterations."""
     path = os.path.join(ROOT, "profiles", f"{kernel_key}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
-    if not m or not d or d.group(1) != source_digest():
+    if not d or d.group(1) != source_digest():
         return None
-    return float(m.group(1))
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if m:
+        return float(m.group(1))
+    m = re.search(r"traffic_bytes_per_iteration:\s*([0-9.eE+]+)", text)
+    if m:
+        return float(m.group(1)) * iters_per_launch
+    return None
 
 
 def measured_hbm_peak():
@@ -94,14 +102,47 @@ def measured_hbm_peak():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and throttle reasons sampled during the timed region.
+
+    NVML (read-only queries) from a thread every 5 ms, so that timed regions of
+    a few tens of milliseconds still get samples; nvidia-smi at 200 ms when
+    NVML cannot be used."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
+        import threading
         self.proc = None
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+
+            def run():
+                while not self.stop_evt.is_set():
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                             int(reasons_fn(h))))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(0.005)
+            self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx, int(reasons_fn(h))))
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
@@ -111,6 +152,16 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            sm = [float(a) for a, _, _ in self.samples]
+            mx = [float(b) for _, b, _ in self.samples]
+            reasons = {name for _, _, r in self.samples for name, bit in self.BITS.items() if r & bit}
+            if not sm:
+                return None
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                    "reasons": sorted(reasons), "source": "nvml"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -136,7 +187,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+                "reasons": sorted(reasons), "source": "nvidia-smi"}
 
 
 _WORKLOAD = {}
@@ -477,7 +528,7 @@ def main():
             variant = "persistent grid, x, r, M^-1 on chip"
         else:
             variant = "persistent grid, vectors in HBM"
-        traffic = profile_traffic(f"cg_kernel_{args.workload}_{args.dtype}")
+        traffic = profile_traffic(f"cg_kernel_{args.workload}_{args.dtype}", (fwd_it + adj_it) / 2)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
                 "kernel": f"PCG solve kernel ({variant}), one launch per solve",
