@@ -132,6 +132,10 @@ __device__ __forceinline__ void system_sums_dyn(const double *const *arr, int nt
     block_sums<NT, NV>(out, red);
 }
 
+__device__ __forceinline__ void red_release_gpu_u32(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Device-wide barrier on a monotonically increasing arrival counter: the k-th
 // barrier of the launch completes when the counter reaches k * gridDim.x, a
 // target every block knows, so arrival is a single fire-and-forget add and the
@@ -148,8 +152,10 @@ __device__ __forceinline__ bool grid_sync(unsigned *sync, unsigned &target, long
     if (threadIdx.x == 0) {
         unsigned *count = sync, *err = sync + 2;
         int ok = 1;
-        __threadfence();
-        atomicAdd(count, 1u);
+        // The arrival is a release at gpu scope: it orders every write of the
+        // block (ordered before it by the block barrier above) before the
+        // count; the polls below are acquires, so no separate fences are needed.
+        red_release_gpu_u32(count, 1u);
         const unsigned long long t0 = global_timer_ns();
         unsigned spins = 0;
         while ((int)(ld_acquire_u32(count) - target) < 0) {
@@ -163,7 +169,6 @@ __device__ __forceinline__ bool grid_sync(unsigned *sync, unsigned &target, long
             }
         }
         if (ok && ld_acquire_u32(err) != 0) ok = 0;
-        __threadfence();
         if (watch) *watched = ld_acquire_u32(watch);
         *flag = ok;
     }
@@ -513,8 +518,7 @@ cg_grid_kernel(CgArgs<T> a) {
             __syncthreads();
             if (tid == 0) {
                 if (tile_flags && go_on) {
-                    __threadfence();
-                    st_release_u32(a.pflag + tt, (unsigned)k);
+                    st_release_u32(a.pflag + tt, (unsigned)k);   // release: the tile's p first
                 }
                 if (go_on) {
                     l_rho[lt] = rho_new;
