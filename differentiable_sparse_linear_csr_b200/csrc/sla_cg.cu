@@ -136,6 +136,40 @@ __device__ __forceinline__ void red_release_gpu_u32(unsigned *p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// grid_sync in two halves, for work that needs neither the barrier's partials
+// nor other blocks' writes: grid_arrive announces the block (after a block
+// barrier) and grid_wait completes the barrier.  Every block calls both, in
+// this order, with nothing between them that other blocks wait for.
+__device__ __forceinline__ void grid_arrive(unsigned *sync, unsigned &target) {
+    __syncthreads();
+    target += gridDim.x;
+    if (threadIdx.x == 0) red_release_gpu_u32(sync, 1u);
+}
+
+__device__ __forceinline__ bool grid_wait(unsigned *sync, unsigned target, long long timeout_ns, int *flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned *count = sync, *err = sync + 2;
+        int ok = 1;
+        const unsigned long long t0 = global_timer_ns();
+        unsigned spins = 0;
+        while ((int)(ld_acquire_u32(count) - target) < 0) {
+            if ((spins++ & 7u) == 0) {
+                if (ld_acquire_u32(err) != 0) { ok = 0; break; }
+                if ((long long)(global_timer_ns() - t0) > timeout_ns) {
+                    atomicExch(err, 1u);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        if (ok && ld_acquire_u32(err) != 0) ok = 0;
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
 // Device-wide barrier on a monotonically increasing arrival counter: the k-th
 // barrier of the launch completes when the counter reaches k * gridDim.x, a
 // target every block knows, so arrival is a single fire-and-forget add and the
@@ -472,9 +506,31 @@ cg_grid_kernel(CgArgs<T> a) {
                 l_alpha[lt] = alpha;
             }
         }
-        if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
+        // x += alpha p needs neither beta nor other blocks: it runs while the
+        // barrier completes
+        grid_arrive(a.sync, target);
+        for (int lt = 0; lt < nlt; ++lt) {
+            if (l_state[lt] != kActive) continue;
+            const int tile = blockIdx.x + lt * G;
+            const int s = tile / a.ntiles, tt = tile % a.ntiles;
+            const T al = (T)l_alpha[lt];
+            const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
+            const T *pg = a.p + (int64_t)s * n;
+            if constexpr (ONCHIP) {
+#pragma unroll
+                for (int j = 0; j < RPT; ++j) {
+                    const int i = r0 + tid + j * NT;
+                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * pg[i];
+                }
+            } else {
+                T *xg = a.x + (int64_t)s * n;
+#pragma unroll 4
+                for (int i = r0 + tid; i < r1; i += NT) xg[i] = xg[i] + al * pg[i];
+            }
+        }
+        if (!grid_wait(a.sync, target, a.timeout_ns, &flag)) { give_up(a); return; }
 
-        // ---- phase C: x += alpha p; stopping test; beta; p = z + beta p
+        // ---- phase C: stopping test; beta; p = z + beta p
         for (int lt = 0; lt < nlt; ++lt) {
             if (l_state[lt] != kActive) continue;
             const int tile = blockIdx.x + lt * G;
@@ -490,29 +546,21 @@ cg_grid_kernel(CgArgs<T> a) {
             else if (!a.fixed && sqrt(rr) <= tol) st = SLA_CONVERGED;
             else if (rr == 0.0) st = SLA_CONVERGED;
             else if (k >= a.limit) st = a.fixed ? SLA_FIXED_DONE : SLA_NOT_CONVERGED;
-            const T al = (T)l_alpha[lt];
             const T bt = (T)(rho_new / l_rho[lt]);
             const bool go_on = st == kActive;
             const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
             T *pg = a.p + (int64_t)s * n;
-            if constexpr (ONCHIP) {
+            if (go_on) {
+                if constexpr (ONCHIP) {
 #pragma unroll
-                for (int j = 0; j < RPT; ++j) {
-                    const int i = r0 + tid + j * NT;
-                    if (i < r1) {
-                        const T pi = pg[i];
-                        xs_[i - r0] = xs_[i - r0] + al * pi;
-                        if (go_on) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pi;
+                    for (int j = 0; j < RPT; ++j) {
+                        const int i = r0 + tid + j * NT;
+                        if (i < r1) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pg[i];
                     }
-                }
-            } else {
-                T *xg = a.x + (int64_t)s * n;
-                const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                } else {
+                    const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
 #pragma unroll 4
-                for (int i = r0 + tid; i < r1; i += NT) {
-                    const T pi = pg[i];
-                    xg[i] = xg[i] + al * pi;
-                    if (go_on) pg[i] = dg[i] * rg[i] + bt * pi;
+                    for (int i = r0 + tid; i < r1; i += NT) pg[i] = dg[i] * rg[i] + bt * pg[i];
                 }
             }
             __syncthreads();
