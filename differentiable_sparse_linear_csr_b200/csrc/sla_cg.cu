@@ -62,6 +62,7 @@ struct CgArgs {
     unsigned *pflag;                        // [ntiles] iteration whose p a tile has written
     const int32_t *sell_ptr, *sell_cols;   // sliced layout of the pattern (SELL kernels)
     const T *sell_vals;                     // [B][sell_nnz] values in that layout
+    const SellRec<T> *sell_rec;             // or [B][sell_nnz] value-and-column records
     int64_t sell_nnz;
 };
 
@@ -409,14 +410,27 @@ cg_grid_kernel(CgArgs<T> a) {
             const T *pg = a.p + (int64_t)s * n;
             double acc[1] = {0.0};
             if constexpr (ONCHIP && SELL) {
-                const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
+                if (a.sell_rec) {
+                    const SellRec<T> *rec = a.sell_rec + (int64_t)s * a.sell_nnz;
 #pragma unroll
-                for (int j = 0; j < RPT; ++j) {
-                    const int i = r0 + tid + j * NT;
-                    if (i < r1) {
-                        const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i);
-                        qreg[j] = qi;
-                        acc[0] += (double)pg[i] * (double)qi;
+                    for (int j = 0; j < RPT; ++j) {
+                        const int i = r0 + tid + j * NT;
+                        if (i < r1) {
+                            const T qi = sell_row_rec<false>(a.sell_ptr, rec, pg, i);
+                            qreg[j] = qi;
+                            acc[0] += (double)pg[i] * (double)qi;
+                        }
+                    }
+                } else {
+                    const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
+#pragma unroll
+                    for (int j = 0; j < RPT; ++j) {
+                        const int i = r0 + tid + j * NT;
+                        if (i < r1) {
+                            const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i);
+                            qreg[j] = qi;
+                            acc[0] += (double)pg[i] * (double)qi;
+                        }
                     }
                 }
             } else if constexpr (ONCHIP) {
@@ -430,12 +444,21 @@ cg_grid_kernel(CgArgs<T> a) {
                     }
                 }
             } else if constexpr (SELL) {
-                const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
                 T *qg = a.q + (int64_t)s * n;
-                for (int i = r0 + tid; i < r1; i += NT) {
-                    const T qi = sell_row<true>(a.sell_ptr, a.sell_cols, svals, pg, i);
-                    qg[i] = qi;
-                    acc[0] += (double)pg[i] * (double)qi;
+                if (a.sell_rec) {
+                    const SellRec<T> *rec = a.sell_rec + (int64_t)s * a.sell_nnz;
+                    for (int i = r0 + tid; i < r1; i += NT) {
+                        const T qi = sell_row_rec<true>(a.sell_ptr, rec, pg, i);
+                        qg[i] = qi;
+                        acc[0] += (double)pg[i] * (double)qi;
+                    }
+                } else {
+                    const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
+                    for (int i = r0 + tid; i < r1; i += NT) {
+                        const T qi = sell_row<true>(a.sell_ptr, a.sell_cols, svals, pg, i);
+                        qg[i] = qi;
+                        acc[0] += (double)pg[i] * (double)qi;
+                    }
                 }
             } else {
                 T *qg = a.q + (int64_t)s * n;
@@ -1181,6 +1204,23 @@ cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, 
             }
         }
         if (!grid_sync(a.sync, target, a.timeout_ns, &flag)) { give_up_il(); return; }
+    }
+}
+
+// The sliced layout's value-and-column records of every system.
+template <typename T>
+__global__ void sell_pack_kernel(int64_t sell_nnz, int64_t nnz, int B, const int32_t *__restrict__ map,
+                                 const int32_t *__restrict__ cols, const T *__restrict__ vals,
+                                 SellRec<T> *__restrict__ out) {
+    const int64_t slot = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (slot >= sell_nnz) return;
+    const int t = map[slot];
+    const int c = cols[slot];
+    for (int b = 0; b < B; ++b) {
+        SellRec<T> r{};
+        r.v = t >= 0 ? vals[(int64_t)b * nnz + t] : T(0);
+        r.c = c;
+        out[(int64_t)b * sell_nnz + slot] = r;
     }
 }
 
@@ -1944,7 +1984,7 @@ static size_t cg_ws_bytes(const Csr *h, bool adjoint) {
     const size_t B = h->batch, n = h->n_rows, ntot = B * (size_t)h->ntiles;
     size_t b = align_up(64) + align_up(4 * B * 8) + align_up(B * 4) + align_up(4 * ntot * 8);
     b += 4 * align_up(B * n * ts);
-    if (h->has_sell) b += align_up(B * (size_t)h->sell_nnz * ts);
+    if (h->has_sell) b += align_up(B * (size_t)h->sell_nnz * (ts == 8 ? 16 : 8));   // values or records
     b += align_up((size_t)h->ntiles * 4);   // p-ready flags
     if (h->il_blocks > 0)                   // interleaved x and b, tile partials
         b += 2 * align_up(B * n * ts) + align_up(4 * B * (size_t)h->il_blocks * 8);
@@ -2082,13 +2122,23 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             return SLA_OK;
         }
         if (sell) {
-            T *sv = c.take<T>((size_t)a.B * h->sell_nnz);
-            sla_status st = sell_values(h, vals, sv, s);
-            if (st != SLA_OK) return st;
             a.sell_ptr = h->sell_ptr;
             a.sell_cols = h->sell_cols;
-            a.sell_vals = sv;
             a.sell_nnz = h->sell_nnz;
+            const char *pk = getenv("SLA_SELL_PACK");
+            const bool pack = pk && pk[0] == '1' && !(h->grid2 && a.B == 1);
+            if (pack) {
+                SellRec<T> *rec = c.take<SellRec<T>>((size_t)a.B * h->sell_nnz);
+                sell_pack_kernel<T><<<(unsigned)((h->sell_nnz + 255) / 256), 256, 0, s>>>(
+                    h->sell_nnz, h->nnz, a.B, h->sell_map, h->sell_cols, vals, rec);
+                SLA_CHECK_LAUNCH();
+                a.sell_rec = rec;
+            } else {
+                T *sv = c.take<T>((size_t)a.B * h->sell_nnz);
+                sla_status st = sell_values(h, vals, sv, s);
+                if (st != SLA_OK) return st;
+                a.sell_vals = sv;
+            }
         }
         SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
         if (a.pflag) SLA_CHECK_CUDA(cudaMemsetAsync(a.pflag, 0, (size_t)h->ntiles * sizeof(unsigned), s));

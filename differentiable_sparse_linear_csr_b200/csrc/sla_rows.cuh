@@ -124,6 +124,52 @@ __device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
     return s;
 }
 
+// A slot of the sliced layout with its value and column in one record, so
+// that one vector load brings both: 8 bytes for fp32, 16 (4 of padding) for fp64.
+template <typename T> struct SellRec;
+template <> struct __align__(16) SellRec<double> { double v; int32_t c, pad; };
+template <> struct __align__(8) SellRec<float> { float v; int32_t c; };
+
+template <bool STREAM, typename T>
+__device__ __forceinline__ void sell_rec_load(const SellRec<T> *p, T &v, int &c) {
+    if constexpr (sizeof(T) == 8) {
+        int4 u;
+        if constexpr (STREAM)
+            asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "l"(p));
+        else
+            u = __ldg(reinterpret_cast<const int4 *>(p));
+        v = __hiloint2double(u.y, u.x);
+        c = u.z;
+    } else {
+        int2 u;
+        if constexpr (STREAM)
+            asm volatile("ld.global.nc.L1::no_allocate.v2.s32 {%0,%1}, [%2];" : "=r"(u.x), "=r"(u.y) : "l"(p));
+        else
+            u = __ldg(reinterpret_cast<const int2 *>(p));
+        v = __int_as_float(u.x);
+        c = u.y;
+    }
+}
+
+// sell_row over packed records: same entries, order and rounding.
+template <bool STREAM, typename T>
+__device__ __forceinline__ T sell_row_rec(const int32_t *__restrict__ sptr, const SellRec<T> *__restrict__ rec,
+                                          const T *v, int i) {
+    const int sl = i / kSellRows;
+    const int b0 = __ldg(sptr + sl);
+    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
+    const int base = b0 + i % kSellRows;
+    T s = T(0);
+    for (int k = 0; k < w; ++k) {
+        T a;
+        int c;
+        sell_rec_load<STREAM>(rec + base + k * kSellRows, a, c);
+        s += a * v[c];
+    }
+    return s;
+}
+
 // Row of the sliced layout times the direction p_k = z + beta p_prev, formed
 // per gathered entry with one fused multiply-add (the owner of each row forms
 // the same value the same way from its own M^-1 r, rounded once, as z).

@@ -130,7 +130,9 @@ typedef struct {
                                  the two-barrier form (directions formed while gathered);
                                  the environment variables SLA_GRID_ONCHIP=0 and
                                  SLA_GRID2=0, read at creation, turn these variants off */
-    int32_t grid_tile_rows;   /* rows of one grid-solver tile */
+    int32_t grid_tile_rows;   /* rows of one grid-solver tile (SLA_SELL_PACK=1, read at each
+                                 solve, makes the sliced SpMV read value-and-column records,
+                                 one load an entry; off by default, see the design notes) */
     int32_t sliced;           /* 1 if the grid solver uses the 8-row sliced layout (one
                                  extra value-gather kernel per solve) */
     int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
