@@ -84,3 +84,54 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "_LIB_PATH", str(tmp_path / "libsla.so"))
     with pytest.raises(ImportError, match="missing"):
         L.lib()
+
+
+def _header_struct_fields(name):
+    """(type, field) pairs of a `typedef struct { ... } name;` in include/sla.h."""
+    src = open(os.path.join(ROOT, "include", "sla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    m = re.search(r"typedef struct\s*\{([^}]*)\}\s*" + name + r"\s*;", src)
+    assert m, name
+    out = []
+    for decl in m.group(1).split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        parts = decl.split()
+        ctype, names = parts[0], " ".join(parts[1:])
+        for n in names.split(","):
+            n = n.strip().lstrip("*")
+            out.append((ctype, n))
+    return out
+
+
+_CTYPES = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "double": ctypes.c_double}
+
+
+@pytest.mark.parametrize("name,mirror", [("sla_csr_props", "sla_csr_props"), ("sla_cg_opts", "sla_cg_opts")])
+def test_ctypes_mirrors_match_the_header(name, mirror):
+    """Field names, order and types of the binding's structures are the header's,
+    so the two sides agree on the layout."""
+    hdr = _header_struct_fields(name)
+    fields = getattr(L, mirror)._fields_
+    assert [n for _, n in hdr] == [f[0] for f in fields]
+    for (ct, n), (fn, ft) in zip(hdr, fields):
+        assert _CTYPES[ct] == ft, (n, ct, ft)
+
+
+def test_info_struct_is_three_device_pointers():
+    hdr = _header_struct_fields("sla_cg_info")
+    assert [n for _, n in hdr] == [f[0] for f in L.sla_cg_info._fields_] == ["iters", "relres", "status"]
+
+
+def test_list_create_argument_errors_need_no_gpu():
+    lib = L.lib()
+    h = ctypes.c_void_p()
+    assert lib.sla_csr_list_create(0, ctypes.c_void_p(256), 4, 0, ctypes.c_void_p(256), None, 0, 0, None,
+                                   ctypes.byref(h)) == L.SLA_ERR_INVALID
+    assert "n_items" in L.sla_last_error_string() and h.value is None
+    assert lib.sla_csr_list_create(2, None, 4, 0, ctypes.c_void_p(256), None, 0, 0, None,
+                                   ctypes.byref(h)) == L.SLA_ERR_INVALID
+    assert "item_rows" in L.sla_last_error_string()
+    assert lib.sla_csr_list_create(2, ctypes.c_void_p(256), 4, 0, ctypes.c_void_p(256), None, 0, 0, None,
+                                   None) == L.SLA_ERR_INVALID

@@ -1,0 +1,59 @@
+"""Host-side pieces of bench.py, checked without a GPU: the algorithmic-byte
+model against the per-iteration figures of the two-pass model for the
+1024x1024 Poisson (fp64 and fp32) and 128^3 diffusion systems, the rule that
+a committed ncu traffic figure is used only while the library source matches
+it, and clock sampling that degrades to "no samples" without a GPU."""
+import os
+
+import pytest
+
+import bench
+
+
+def test_two_pass_model_bytes():
+    # one sweep of A ((s_v + 4) nnz + 4 (n + 1)) plus 11 vector passes (11 s_v n)
+    assert bench.per_iteration_bytes(1_048_576, 5_238_784, 8) == 159_334_404
+    assert bench.per_iteration_bytes(1_048_576, 5_238_784, 4) == 92_241_924
+    assert bench.per_iteration_bytes(2_097_152, 14_581_760, 8) == 367_919_108
+    # the value gradient reads lambda and x, the pattern, and writes nnz values
+    assert bench.grad_bytes(1_048_576, 5_238_784, 8) == 12 * 5_238_784 + 20 * 1_048_576
+
+
+def _profile(tmp_path, key, body):
+    d = tmp_path / "profiles"
+    d.mkdir(exist_ok=True)
+    (d / f"{key}.md").write_text(body)
+
+
+def test_traffic_is_used_only_for_the_matching_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_digest", lambda: "abc123")
+    _profile(tmp_path, "k_launch", "traffic_bytes_per_launch: 1.5e9\nsource_digest: abc123\n")
+    _profile(tmp_path, "k_iter", "traffic_bytes_per_iteration: 200\nsource_digest: abc123\n")
+    _profile(tmp_path, "k_stale", "traffic_bytes_per_iteration: 200\nsource_digest: ffff00\n")
+    _profile(tmp_path, "k_none", "source_digest: abc123\n")
+    assert bench.profile_traffic("k_launch", 10) == 1.5e9
+    assert bench.profile_traffic("k_iter", 924) == 200 * 924
+    assert bench.profile_traffic("k_stale", 924) is None
+    assert bench.profile_traffic("k_none", 924) is None
+    assert bench.profile_traffic("k_missing", 924) is None
+
+
+def test_source_digest_covers_the_library_source():
+    d = bench.source_digest()
+    assert len(d) == 16 and int(d, 16) >= 0
+    assert d == bench.source_digest()
+
+
+def test_edge_kernel_bytes():
+    m = bench.edge_metrics(n=4, nnz=10, E=3, B=2, vbytes=8, asm_ms=1.0, grad_ms=2.0)
+    assert m["assemble_bytes"] == 4 * 5 + 8 * 10 + 2 * 8 * (3 + 10 + 1)
+    assert m["edge_grad_bytes"] == 8 * 3 + 2 * 8 * (2 * 4 + 3 + 1)
+    assert m["assemble_gbs"] == pytest.approx(m["assemble_bytes"] / 1e-3 / 1e9)
+
+
+def test_clock_sampler_without_a_gpu_returns_nothing():
+    if os.path.exists("/dev/nvidiactl"):
+        pytest.skip("a GPU driver is present")
+    s = bench.ClockSampler(0)
+    assert s.stop() is None
