@@ -12,16 +12,27 @@
 //         z = M^-1 r; beta = r.z / rho; p = z + beta p
 // Dot products accumulate in fp64 for both value types.
 //
-// Two kernels implement it:
+// Kernels, all with the iteration loop on the device and every wait bounded:
 //  * cg_grid_kernel -- one persistent cooperative grid (all blocks resident)
 //    for systems too large for one block.  Rows are split into fixed tiles; a
-//    block owns the same tiles in every phase.  Three device-wide barriers per
-//    iteration separate SpMV+p.q, the x/r update with r.z and r.r, and the
-//    direction update.  Every block reduces the per-tile partials of a system
+//    block owns the same tiles in every phase.  Device-wide barriers separate
+//    SpMV+p.q, the r update with r.z and r.r (x += alpha p runs while the
+//    following barrier completes), and the direction update; for one system
+//    with banded tile dependencies, p-ready tile flags replace the third.
+//    Vectors stay on chip (shared memory and registers) when a block's tile
+//    fits, else in HBM.  Every block reduces the per-tile partials of a system
 //    itself, in one fixed order, so all blocks take identical decisions
 //    without extra communication; results are bit-reproducible run to run.
+//  * cg_grid2_kernel -- the same for one system on chip with two barriers an
+//    iteration: directions are formed while gathered in the next SpMV.
+//  * cg_grid_il_kernel -- batches of 2 or 4 systems in HBM with values and
+//    vectors interleaved by system, one column index for all of them.
 //  * cg_block_kernel -- one thread block per system with x, r, p, q, M^-1 in
 //    shared memory (small systems, large batches): no device-wide barrier.
+//  * cg_cluster_kernel -- one 8-block thread-block cluster per small system,
+//    the matrix slice and vectors in each block's shared memory, p over DSMEM.
+//  * cg_segment_kernel -- lists of systems with their own patterns, one item
+//    a block, largest first.
 #include <cmath>
 #include <cstdlib>
 #include <cooperative_groups.h>

@@ -1,7 +1,8 @@
 // CSR handle: pattern validation, pattern statistics, diagonal positions and
 // (on request) A^T's pattern.  A handle is the shared-pattern `SparseTensor`
 // of the torch-sla summary page (technical summary, "Methodology" 1: one
-// matrix, or a batch of value sets sharing one pattern).
+// matrix, or a batch of value sets sharing one pattern); a list handle holds
+// items with their own patterns, stored block-diagonally (`SparseTensorList`).
 #include <climits>
 #include <cstdlib>
 #include <cstring>

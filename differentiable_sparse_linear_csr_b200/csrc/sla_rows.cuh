@@ -1,7 +1,9 @@
 // Row-parallel building blocks: one row of a CSR matrix times a vector, with
 // LANES threads of a warp cooperating on the row (LANES in 1..32, a power of
-// two).  Matrix arrays are read through the read-only path; the vector is read
-// with plain loads because the persistent solver rewrites it between phases.
+// two), and one row of the sliced layout times a vector (plain, as
+// value-and-column records, or forming the CG direction while gathering).
+// Matrix arrays are read through the read-only path; the vector is read with
+// plain loads because the persistent solver rewrites it between phases.
 #pragma once
 
 #include <type_traits>
