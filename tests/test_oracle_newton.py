@@ -9,7 +9,6 @@ case kappa = 0, quadratic convergence of the residual norms, and central finite
 differences of L = 0.5 ||u - u_obs||^2 in f and kappa through dense Newton.
 """
 import numpy as np
-import pytest
 
 from differentiable_sparse_linear_csr_b200 import workloads as W
 from oracle import oracle as O
