@@ -106,7 +106,8 @@ typedef struct {
     int32_t reserved;         /* must be 0 */
 } sla_cg_opts;
 
-/* Per-system outputs, device pointers to [B] arrays; any may be NULL. */
+/* Per-system outputs, device pointers to [B] arrays ([n_items] for a list
+ * handle, see sla_csr_list_create); any may be NULL. */
 typedef struct {
     int32_t *iters;           /* completed iterations (alpha-updates) */
     double *relres;           /* recursive ||r_k|| / ||b|| at exit */
