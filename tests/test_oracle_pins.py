@@ -11,6 +11,7 @@ The method: Jacobi-preconditioned CG and its implicit-function-theorem adjoint
 from "torch-sla: Differentiable Sparse Linear Algebra with Adjoint Solvers and
 Sparse Tensor Parallelism for PyTorch" (technical summary, "Methodology" 1-2).
 """
+import ctypes
 import math
 import os
 from fractions import Fraction
@@ -75,6 +76,97 @@ def test_worked_2x2_iterates_and_gradient():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype", [np.float64, np.float32])
+
+def _fp32_example():
+    g = _golden("pcg_fp32_policy_3x3.txt")
+    rp = np.array([int(f) for f in g["rowptr"]], np.int32)
+    ci = np.array([int(f) for f in g["colind"]], np.int32)
+    v = np.array([float(f) for f in g["values"]], np.float32)
+    b = np.array([float(f) for f in g["b"]], np.float32)
+    # the stored iterates are fp32 numbers; float() of the exact fraction is exact
+    x1 = np.array([float(f) for f in g["x1"]], np.float32)
+    x2 = np.array([float(f) for f in g["x2"]], np.float32)
+    assert all(float(np.float32(float(f))) == f for f in g["x1"] + g["x2"])
+    return rp, ci, v, b, x1, x2
+
+
+def test_fp32_precision_policy_worked_example_bit_for_bit():
+    """The fp32 oracle reproduces the hand-worked iterates of the 3x3 example
+    exactly: every rounding of the stated precision policy is where the
+    derivation puts it."""
+    rp, ci, v, b, x1, x2 = _fp32_example()
+    for k, want in ((1, x1), (2, x2)):
+        x, info = O.pcg(rp, ci, v, b, fixed_iters=k)
+        assert x.dtype == np.float32 and info.iters[0] == k
+        assert np.array_equal(x.view(np.uint32), want.view(np.uint32)), (k, x, want)
+
+
+# Slips in the fp32 arithmetic that a plausible implementation could make, as
+# textual changes of the oracle's source (applied to a copy built on the side).
+_FP32_SLIPS = {
+    "dots accumulated in fp32": [
+        ("    double s = 0.0;\n    if (!reverse) {\n        for (int32_t i = 0; i < n; ++i) s = s + (double)a[i] * (double)b[i];\n"
+         "    } else {\n        for (int32_t i = n - 1; i >= 0; --i) s = s + (double)a[i] * (double)b[i];",
+         "    T s = (T)0;\n    if (!reverse) {\n        for (int32_t i = 0; i < n; ++i) s = s + a[i] * b[i];\n"
+         "    } else {\n        for (int32_t i = n - 1; i >= 0; --i) s = s + a[i] * b[i];")],
+    "alpha kept in fp64 in the x and r updates": [
+        ("x[i] = x[i] + a * p[i];", "x[i] = x[i] + alpha * p[i];"),
+        ("r[i] = r[i] - a * q[i];", "r[i] = r[i] - alpha * q[i];")],
+    "beta kept in fp64 in the direction update": [
+        ("p[i] = q[i] + bt * p[i];", "p[i] = q[i] + beta * p[i];")],
+    "matrix rows summed in fp64": [
+        ("        T s = (T)0;\n        if (!reverse) {\n            for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t)\n"
+         "                s = s + vals[t] * x[colind[t]];",
+         "        double s = 0.0;\n        if (!reverse) {\n            for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t)\n"
+         "                s = s + (double)vals[t] * (double)x[colind[t]];")],
+}
+
+
+def _oracle_variant(tmp_path, edits):
+    """liboracle built from a copy of the oracle's source with `edits` applied."""
+    import shutil
+    import subprocess
+    src_dir = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle")
+    for f in ("oracle.c", "oracle_body.h"):
+        shutil.copy(os.path.join(src_dir, f), tmp_path / f)
+    body = (tmp_path / "oracle_body.h").read_text()
+    for old, new in edits:
+        assert body.count(old) == 1, old
+        body = body.replace(old, new)
+    (tmp_path / "oracle_body.h").write_text(body)
+    so = tmp_path / "liboracle_variant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-o", str(so), str(tmp_path / "oracle.c"), "-lm"])
+    lib = ctypes.CDLL(str(so))
+    P, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.orc_pcg_f32.argtypes = [i32, P, P, P, P, P, P, P]
+    lib.orc_pcg_f32.restype = i32
+    return lib
+
+
+def _variant_pcg_f32(lib, rp, ci, v, b, k):
+    x = np.zeros(b.shape[0], np.float32)
+    o = O._Opts(0.0, 0.0, k, k, 1, 0, 0)
+    r = O._Result()
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    assert lib.orc_pcg_f32(b.shape[0], p(rp), p(ci), p(v), p(b), p(x), ctypes.byref(o), ctypes.byref(r)) == 0
+    return x
+
+
+@pytest.mark.parametrize("slip", sorted(_FP32_SLIPS))
+def test_fp32_worked_example_catches_a_planted_slip(slip, tmp_path):
+    """Each slip, planted in a copy of the oracle, changes the worked example's
+    second iterate, so the bit-for-bit pin above would fail on it; the copy
+    without edits reproduces the example."""
+    rp, ci, v, b, x1, x2 = _fp32_example()
+    (tmp_path / "clean").mkdir()
+    (tmp_path / "slip").mkdir()
+    clean = _oracle_variant(tmp_path / "clean", [])
+    assert np.array_equal(_variant_pcg_f32(clean, rp, ci, v, b, 2).view(np.uint32), x2.view(np.uint32))
+    lib = _oracle_variant(tmp_path / "slip", _FP32_SLIPS[slip])
+    x = _variant_pcg_f32(lib, rp, ci, v, b, 2)
+    assert not np.array_equal(x.view(np.uint32), x2.view(np.uint32)), slip
+
 def test_spmv_matches_dense_product(dtype):
     rng = np.random.default_rng(11)
     for n_rows, n_cols in [(1, 1), (7, 13), (60, 40), (200, 200)]:
