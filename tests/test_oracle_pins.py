@@ -71,12 +71,6 @@ def test_worked_2x2_iterates_and_gradient():
     np.testing.assert_allclose(G, [float(f) for f in g["grad_values"]], rtol=1e-14, atol=0)
 
 
-# ---------------------------------------------------------------------------
-# SpMV and dense LU against numpy
-# ---------------------------------------------------------------------------
-
-@pytest.mark.parametrize("dtype", [np.float64, np.float32])
-
 def _fp32_example():
     g = _golden("pcg_fp32_policy_3x3.txt")
     rp = np.array([int(f) for f in g["rowptr"]], np.int32)
@@ -105,10 +99,11 @@ def test_fp32_precision_policy_worked_example_bit_for_bit():
 # textual changes of the oracle's source (applied to a copy built on the side).
 _FP32_SLIPS = {
     "dots accumulated in fp32": [
-        ("    double s = 0.0;\n    if (!reverse) {\n        for (int32_t i = 0; i < n; ++i) s = s + (double)a[i] * (double)b[i];\n"
-         "    } else {\n        for (int32_t i = n - 1; i >= 0; --i) s = s + (double)a[i] * (double)b[i];",
-         "    T s = (T)0;\n    if (!reverse) {\n        for (int32_t i = 0; i < n; ++i) s = s + a[i] * b[i];\n"
-         "    } else {\n        for (int32_t i = n - 1; i >= 0; --i) s = s + a[i] * b[i];")],
+        ("    double s = 0.0;\n    if (!reverse) {\n", "    T s = (T)0;\n    if (!reverse) {\n"),
+        ("        for (int32_t i = 0; i < n; ++i) s = s + (double)a[i] * (double)b[i];\n",
+         "        for (int32_t i = 0; i < n; ++i) s = s + a[i] * b[i];\n"),
+        ("        for (int32_t i = n - 1; i >= 0; --i) s = s + (double)a[i] * (double)b[i];",
+         "        for (int32_t i = n - 1; i >= 0; --i) s = s + a[i] * b[i];")],
     "alpha kept in fp64 in the x and r updates": [
         ("x[i] = x[i] + a * p[i];", "x[i] = x[i] + alpha * p[i];"),
         ("r[i] = r[i] - a * q[i];", "r[i] = r[i] - alpha * q[i];")],
@@ -167,6 +162,12 @@ def test_fp32_worked_example_catches_a_planted_slip(slip, tmp_path):
     x = _variant_pcg_f32(lib, rp, ci, v, b, 2)
     assert not np.array_equal(x.view(np.uint32), x2.view(np.uint32)), slip
 
+# ---------------------------------------------------------------------------
+# SpMV and dense LU against numpy
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("dtype", [np.float64, np.float32])
 def test_spmv_matches_dense_product(dtype):
     rng = np.random.default_rng(11)
     for n_rows, n_cols in [(1, 1), (7, 13), (60, 40), (200, 200)]:
