@@ -93,6 +93,15 @@ def profile_traffic(kernel_key: str, iters_per_launch: float):
     return None
 
 
+def profile_metric(kernel_key: str, name: str):
+    """A named figure (`name: value`) from a committed ncu summary, or None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_key}.md")
+    if not os.path.exists(path):
+        return None
+    m = re.search(rf"^{re.escape(name)}:\s*([0-9.eE+-]+)", open(path).read(), re.M)
+    return float(m.group(1)) if m else None
+
+
 def measured_hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -197,6 +206,17 @@ CPU_ITERS = {"c1": 1000, "c2": 300, "c3": 100, "c4": 2000, "c5": 12, "c5rcm": 12
              "c3b4": 100}
 
 
+def split_workload(w, world: int, rank: int):
+    """Rank `rank`'s contiguous shard of the batch of `w` (the same batch on
+    every rank; see sharding.shard_range)."""
+    import dataclasses
+    from differentiable_sparse_linear_csr_b200.sharding import shard_range
+    lo, hi = shard_range(w.batch, world, rank)
+    return dataclasses.replace(
+        w, values=w.values[lo:hi], b=w.b[lo:hi], xstar=w.xstar[lo:hi],
+        weights=None if w.weights is None else w.weights[lo:hi])
+
+
 def load_workload(name: str, rank: int = 0):
     """The synthetic workload `name`; every rank gets its own seed (replicas)."""
     from differentiable_sparse_linear_csr_b200 import workloads as W
@@ -245,7 +265,7 @@ def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2", edges: bool =
                             fixed_iters=k_iters)
         O.grad_values(rp, ci, lam, x)
         dt = time.perf_counter() - t0
-        return 2 * 32 * k_iters / dt, dt
+        return 2 * 32 * k_iters / dt, dt, x
     t0 = time.perf_counter()
     if edges:
         v = O.laplacian_assemble(w.rowptr, w.colind, w.edges[0], w.edges[1],
@@ -256,7 +276,45 @@ def oracle_sample(dtype_name: str, k_iters: int, name: str = "c2", edges: bool =
     if edges:
         O.laplacian_grad_values(w.rowptr, w.colind, w.edges[0], w.edges[1], G)
     dt = time.perf_counter() - t0
-    return 2 * k_iters / dt, dt
+    return 2 * k_iters / dt, dt, x
+
+
+def host_cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_all_cores(args, k: int, x_single):
+    """The same oracle sample with the oracle's source built with OpenMP, on
+    every core this process may use, in a child process; its forward solution
+    is checked against the single-threaded one to the parity tolerance (only
+    the order of the dot products' additions differs)."""
+    import tempfile
+    import numpy as np
+    cores = len(os.sched_getaffinity(0))
+    with tempfile.TemporaryDirectory() as tmp:
+        out = os.path.join(tmp, "x.npy")
+        code = (f"import sys, json, numpy as np; sys.path.insert(0, {ROOT!r}); import bench; "
+                f"r, t, x = bench.oracle_sample({args.dtype!r}, {k}, {args.workload!r}, {bool(args.edges)}); "
+                f"np.save({out!r}, x); print(json.dumps([r, t]))")
+        env = dict(os.environ, SLA_ORACLE_OPENMP="1", OMP_NUM_THREADS=str(cores), OMP_PROC_BIND="close")
+        res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                             timeout=900)
+        if res.returncode != 0:
+            return {"error": res.stderr.strip().splitlines()[-1:] or ["failed"]}
+        rate, secs = json.loads(res.stdout.strip().splitlines()[-1])
+        x_omp = np.load(out)
+    xs = np.asarray(x_single, np.float64)
+    err = float(np.linalg.norm(np.asarray(x_omp, np.float64) - xs) / max(np.linalg.norm(xs), 1e-300))
+    tol = 1e-8 if args.dtype == "f64" else 1e-4
+    return {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle, OpenMP build of the same source",
+            "cpu_model": host_cpu_model(), "seconds": secs,
+            "x_rel_diff_vs_single_thread": err, "within_parity_tolerance": err <= tol}
 
 
 def reduce_over_ranks(total_ms: float, iters_per_step: float, device):
@@ -275,6 +333,134 @@ def reduce_over_ranks(total_ms: float, iters_per_step: float, device):
     return float(t.item()), float(w.item())
 
 
+def spmv_bytes(n: int, nnz: int, vbytes: int) -> int:
+    """One y = A x: the matrix once ((vbytes + 4) nnz + 4 (n + 1)), x once (ideal
+    gather) and y written once."""
+    return (vbytes + 4) * nnz + 4 * (n + 1) + 2 * vbytes * n
+
+
+def time_kernel_ms(fn, flush, reps: int = 20, warmup: int = 3) -> float:
+    """Mean CUDA-event time of fn() on the current stream, L2 flushed (outside
+    the events) before every launch."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    total = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / reps
+
+
+def spmv_block(A, vals, n: int, nnz: int, B: int, vbytes: int, dt, dev, flush, peak: float) -> dict:
+    """The standalone `.matvec` (sla_spmv, y = A x) on the workload's matrix."""
+    import torch
+    from differentiable_sparse_linear_csr_b200 import _lib as L
+    x = torch.linspace(-1.0, 1.0, B * n, dtype=dt, device=dev).reshape(B, n)
+    y = torch.empty(B, n, dtype=dt, device=dev)
+    ms = time_kernel_ms(lambda: L.sla_spmv(A.handle, vals, x, y, 0, 1.0, 0.0), flush)
+    by = spmv_bytes(n, nnz, vbytes) * B
+    gbs = by / (ms / 1000.0) / 1e9
+    return {"ms": ms, "algorithmic_bytes": by, "gbs": gbs, "frac_of_hbm_peak": gbs / peak,
+            "kernel": "sla_spmv (one-thread rows: 256-row chunks staged in shared memory)"}
+
+
+def l2_stream_peak_gbs(dev) -> float:
+    """Read bandwidth of an L2-resident 48 MB buffer (a plain torch reduction,
+    repeated), as the denominator of kernels whose working set stays in L2."""
+    import torch
+    buf = torch.ones(6 << 20, dtype=torch.float64, device=dev)     # 48 MB < 126 MB L2
+    out = torch.empty((), dtype=torch.float64, device=dev)
+    for _ in range(5):
+        torch.sum(buf, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 50
+    e0.record()
+    for _ in range(reps):
+        torch.sum(buf, out=out)
+    e1.record()
+    e1.synchronize()
+    return buf.numel() * 8 * reps / (e0.elapsed_time(e1) / 1000.0) / 1e9
+
+
+def secondary_workload(args, name: str, dev, flush, peak: float, peak_kind: str) -> dict:
+    """The HBM-streaming 3-D diffusion workload measured beside the headline:
+    the same step (forward PCG, g = x - x*, adjoint, value gradient), timed the
+    same way, with its solve kernel's roofline and its standalone SpMV."""
+    import torch
+    import differentiable_sparse_linear_csr_b200 as sla
+    from differentiable_sparse_linear_csr_b200 import _lib as L
+    w = load_workload(name)
+    dt = torch.float64 if args.dtype == "f64" else torch.float32
+    vbytes = 8 if args.dtype == "f64" else 4
+    n, nnz, B = w.n, w.nnz, w.batch
+    A = sla.CSR(torch.from_numpy(w.rowptr).to(dev), torch.from_numpy(w.colind).to(dev),
+                batch=B, dtype=dt, symmetric=True)
+    vals = torch.from_numpy(w.values).to(dev, dt).contiguous()
+    b = torch.from_numpy(w.b).to(dev, dt).contiguous()
+    xs = torch.from_numpy(w.xstar).to(dev, dt).contiguous()
+    x, g, lam = (torch.empty(B, n, dtype=dt, device=dev) for _ in range(3))
+    G = torch.empty(B, nnz, dtype=dt, device=dev)
+    fi = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    ai = [torch.empty(B, dtype=t, device=dev) for t in (torch.int32, torch.float64, torch.int32)]
+    ws = torch.empty(L.sla_workspace_bytes(A.handle, L.SLA_OP_ADJOINT), dtype=torch.uint8, device=dev)
+    opts = L.make_opts(rtol=w.rtol, fixed_iters=w.fixed_iters)
+    stream = torch.cuda.current_stream()
+    evs = []
+    for k in range(args.warmup + args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e[0].record(stream)
+        L.sla_cg_solve(A.handle, vals, b, x, opts, L.make_info(*fi), ws)
+        e[1].record(stream)
+        torch.sub(x, xs, out=g)
+        e[2].record(stream)
+        L.sla_cg_adjoint(A.handle, vals, g, lam, opts, L.make_info(*ai), ws)
+        e[3].record(stream)
+        L.sla_grad_values(A.handle, lam, x, G, 0)
+        e[4].record(stream)
+        if k >= args.warmup:
+            evs.append(e)
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(e[0].elapsed_time(e[4]) for e in evs)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    solve_ms = fwd_ms + statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    grad_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+    fwd_it, adj_it = int(fi[0].sum().item()), int(ai[0].sum().item())
+    it_bytes = per_iteration_bytes(n, nnz, vbytes)
+    achieved = (fwd_it + adj_it) * it_bytes / (solve_ms / 1000.0) / 1e9
+    traffic = profile_traffic(f"cg_kernel_{name}_{args.dtype}", (fwd_it + adj_it) / 2)
+    launch_ms = solve_ms / 2
+    out = {"workload": f"{w.description}: forward and adjoint to relative residual {w.rtol:g} "
+                       f"Jacobi-PCG iterations + sparse value gradient",
+           "name": name, "n": n, "nnz": nnz, "value_dtype": args.dtype,
+           "value": (fwd_it + adj_it) / (step_ms / 1000.0), "unit": UNIT,
+           "fwd_adj_grad_ms": step_ms, "forward_ms": fwd_ms, "grad_ms": grad_ms,
+           "forward_iters": fwd_it, "adjoint_iters": adj_it,
+           "statuses": sorted(set(fi[2].tolist()) | set(ai[2].tolist())),
+           "grad_gbs": grad_bytes(n, nnz, vbytes) * B / (grad_ms / 1000.0) / 1e9,
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "peak_source": peak_kind,
+                        "traffic": traffic,
+                        "traffic_gbs": None if traffic is None else traffic / (launch_ms / 1000.0) / 1e9,
+                        "traffic_frac": None if traffic is None else
+                        traffic / (launch_ms / 1000.0) / 1e9 / peak,
+                        "kernel": f"PCG solve kernel (grid_onchip={A.props.grid_onchip}, "
+                                  f"sliced={A.props.sliced}), one launch per solve",
+                        "bytes_per_iteration": it_bytes, "launch_ms": launch_ms},
+           "spmv": spmv_block(A, vals, n, nnz, B, vbytes, dt, dev, flush, peak)}
+    del A
+    return out
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -284,7 +470,7 @@ def run_reference(args):
         oracle_sample(args.dtype, k, args.workload, args.edges)
     total_it, total_t = 0, 0.0
     for _ in range(args.steps):
-        rate, dt = oracle_sample(args.dtype, k, args.workload, args.edges)
+        rate, dt, _ = oracle_sample(args.dtype, k, args.workload, args.edges)
         total_it += rate * dt                     # iterations of the sample (items x 2k for a list)
         total_t += dt
     v = total_it / total_t
@@ -318,7 +504,8 @@ def workload_config(args, w=None):
             "name": args.workload, "n": int(w.n), "nnz": int(w.nnz), "batch": int(w.batch),
             **({"items": int(len(w.item_rows) - 1)} if w.item_rows is not None else {}),
             "value_dtype": args.dtype, "l2": "flushed between steps (write of a 256 MiB buffer)",
-            "parallelism": f"replicas x{world}"}
+            "parallelism": (f"one batch split along its systems x{world}" if getattr(args, "split_batch", False)
+                            else f"replicas x{world}")}
 
 
 def main():
@@ -331,11 +518,19 @@ def main():
     ap.add_argument("--ref-iters", type=int, default=40)
     ap.add_argument("--cpu-iters", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-all-cores", action="store_true",
+                    help="skip the OpenMP build of the oracle on all host cores")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the standalone SpMV and, on the default workload, the 3-D diffusion "
+                         "block measured beside it")
     ap.add_argument("--strategy", type=int, default=0)
     ap.add_argument("--iters", type=int, default=0,
                     help="override the fixed iteration count (short profiler captures)")
     ap.add_argument("--workload", default="c2", choices=WORKLOADS)
+    ap.add_argument("--split-batch", action="store_true",
+                    help="shared-pattern batches (c4, c3b4): the ranks split one batch along the "
+                         "systems instead of each solving its own replica (strong scaling)")
     ap.add_argument("--edges", action="store_true",
                     help="edge-weighted workloads (c3, c4, c5, c5rcm): assemble the values from "
                          "the edge weights and take the gradient back to them")
@@ -364,7 +559,13 @@ def main():
 
     dt = torch.float64 if args.dtype == "f64" else torch.float32
     vbytes = 8 if args.dtype == "f64" else 4
-    w = load_workload(args.workload, rank)
+    if args.split_batch:
+        w_all = load_workload(args.workload, 0)
+        if w_all.item_rows is not None or w_all.batch < world:
+            ap.error(f"--split-batch needs a shared-pattern batch of at least {world} systems")
+        w = split_workload(w_all, world, rank)
+    else:
+        w = load_workload(args.workload, rank)
     n, nnz, B = w.n, w.nnz, w.batch
     fixed = args.iters if args.iters > 0 else w.fixed_iters
     if w.item_rows is not None:
@@ -535,20 +736,43 @@ def main():
                 "algorithmic_bytes_per_launch": (fwd_it + adj_it) * it_bytes / 2,
                 "bytes_per_iteration": it_bytes,
                 "launch_ms": cg_ms / 2}
+        if uses_grid and props.grid_onchip and not props.interleaved:
+            # The on-chip solver keeps x, r, M^-1 in shared memory; the matrix and p
+            # it sweeps every iteration stay in L2 after the first pass, so its
+            # bandwidth roof is L2's, measured here.
+            l2 = l2_stream_peak_gbs(dev)
+            roof.update({"bound": "l2", "peak": l2, "frac": achieved / l2,
+                         "peak_source": "measured in this run: torch reduction over an L2-resident "
+                                        "48 MB buffer",
+                         "hbm_peak": peak, "hbm_peak_source": peak_kind, "frac_of_hbm_peak": achieved / peak,
+                         "ncu_lts_throughput_frac": profile_metric(
+                             f"cg_kernel_{args.workload}_{args.dtype}", "lts_throughput_frac")})
+        spmv = None
+        if w.item_rows is None and not args.no_secondary:
+            spmv = spmv_block(A, vals, n, nnz, B, vbytes, dt, dev, flush, peak)
+        secondary = None
+        if world == 1 and not args.no_secondary and args.workload == "c2" and not args.edges:
+            secondary = secondary_workload(args, "c3", dev, flush, peak, peak_kind)
         gb = grad_bytes(n, nnz, vbytes) * B
-        cpu = None
+        cpu = cpu_all = None
         if not args.no_cpu_baseline and world == 1:
             k = args.cpu_iters if args.cpu_iters > 0 else CPU_ITERS[args.workload]
-            v_cpu, t_cpu = oracle_sample(args.dtype, k, args.workload, args.edges)
+            v_cpu, t_cpu, x_cpu = oracle_sample(args.dtype, k, args.workload, args.edges)
+            sample = (f"{k} forward + {k} adjoint PCG iterations + "
+                      f"{'assembly and edge-weight' if args.edges else 'value'} gradient of "
+                      f"{'the first 32 items' if w.item_rows is not None else 'system 0'}")
             cpu = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
-                   "sample": f"{k} forward + {k} adjoint PCG iterations + "
-                             f"{'assembly and edge-weight' if args.edges else 'value'} gradient of "
-                             f"system 0, single-threaded C ({t_cpu:.1f} s)"}
+                   "cpu_model": host_cpu_model(),
+                   "sample": f"{sample}, single-threaded C ({t_cpu:.1f} s)"}
+            if not args.no_cpu_all_cores:
+                cpu_all = cpu_all_cores(args, k, x_cpu)
+                cpu_all["sample"] = sample
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "strong" if args.split_batch else "weak",
                 "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-                "config": workload_config(args, w),
+                "config": workload_config(args, w_all if args.split_batch else w),
                 "fwd_adj_grad_ms": statistics.mean(step_ms),
                 "forward_ms": statistics.mean(fwd_ms), "adjoint_ms": statistics.mean(adj_ms),
                 "grad_ms": statistics.mean(grad_ms),
@@ -556,7 +780,8 @@ def main():
                 "grad_gbs": None if args.edges else gb / (statistics.mean(grad_ms) / 1000.0) / 1e9,
                 **(edge_metrics(n, nnz, len(w.edges[0]), B, vbytes, statistics.mean(asm_ms),
                                 statistics.mean(grad_ms)) if args.edges else {}),
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roof, "spmv": spmv, "hbm_workload": secondary,
+                "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clock_info}
         print(json.dumps(line), flush=True)

@@ -24,19 +24,26 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _BODY = os.path.join(_HERE, "oracle_body.h")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
 
 CONVERGED, NOT_CONVERGED, BREAKDOWN, NONFINITE, FIXED_DONE = 0, 1, 2, 3, 4
 
 
-def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so next to it (gcc, contraction off)."""
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, contraction off).
+
+    openmp=True builds liboracle_omp.so from the same source with -fopenmp, for
+    the benchmark's all-cores CPU baseline only: rows and vector entries are
+    split over threads (same arithmetic) and dot products are summed per thread
+    before they are combined (another order of the same additions)."""
+    lib = _LIB_OMP if openmp else _LIB
     newest = max(os.path.getmtime(_SRC), os.path.getmtime(_BODY))
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
-        tmp = _LIB + f".tmp{os.getpid()}"
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < newest:
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC",
-                               "-shared", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+                               *(["-fopenmp"] if openmp else []), "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, lib)
+    return lib
 
 
 class _Opts(ctypes.Structure):
@@ -55,9 +62,11 @@ _lib = None
 
 
 def _L():
+    """The oracle library: the single-threaded build, or the OpenMP build when
+    the environment variable SLA_ORACLE_OPENMP=1 is set before first use."""
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = ctypes.CDLL(build(openmp=os.environ.get("SLA_ORACLE_OPENMP") == "1"))
         P = ctypes.c_void_p
         i32, i64 = ctypes.c_int32, ctypes.c_int64
         for sfx in ("f64", "f32"):

@@ -8,6 +8,12 @@
  * to float only where they multiply a float vector.  For T = double everything
  * is double.  Arithmetic is plain C with floating-point contraction disabled at
  * compile time, so every product and sum is rounded separately.
+ *
+ * The OpenMP pragmas are inert in the oracle's own build (compiled without
+ * -fopenmp).  The benchmark's all-cores CPU baseline compiles this same source
+ * with -fopenmp: rows and vector entries are then split over threads, which
+ * changes nothing in their arithmetic, and dot products are summed per thread
+ * and then combined, which changes only the order of their additions.
  */
 
 #define CAT_(a, b) a##_##b
@@ -23,6 +29,7 @@
 void FN(orc_spmv)(int32_t n_rows, const int32_t *rowptr, const int32_t *colind,
                   const T *vals, const T *x, T *y, int32_t reverse)
 {
+    #pragma omp parallel for schedule(static)
     for (int32_t i = 0; i < n_rows; ++i) {
         T s = (T)0;
         if (!reverse) {
@@ -40,6 +47,7 @@ static double FN(dot)(int32_t n, const T *a, const T *b, int32_t reverse)
 {
     double s = 0.0;
     if (!reverse) {
+        #pragma omp parallel for schedule(static) reduction(+:s)
         for (int32_t i = 0; i < n; ++i) s = s + (double)a[i] * (double)b[i];
     } else {
         for (int32_t i = n - 1; i >= 0; --i) s = s + (double)a[i] * (double)b[i];
@@ -84,6 +92,7 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
 
     /* M = diag(A): dinv_i = 1 / A_ii, or 1 without preconditioning. */
     int32_t bad_diag = 0;
+    #pragma omp parallel for schedule(static) reduction(|:bad_diag)
     for (int32_t i = 0; i < n; ++i) {
         T d = (T)0;
         for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t)
@@ -111,8 +120,10 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
     }
     if (opt->x0_given) {
         FN(orc_spmv)(n, rowptr, colind, vals, x, q, rev);
+        #pragma omp parallel for schedule(static)
         for (int32_t i = 0; i < n; ++i) r[i] = b[i] - q[i];
     } else {
+        #pragma omp parallel for schedule(static)
         for (int32_t i = 0; i < n; ++i) r[i] = b[i];
     }
     if (opt->precond && bad_diag) {
@@ -122,6 +133,7 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
         free(r); free(p); free(q); free(dinv);
         return 0;
     }
+    #pragma omp parallel for schedule(static)
     for (int32_t i = 0; i < n; ++i) p[i] = dinv[i] * r[i];
     double rho = FN(dot)(n, r, p, rev);
     double rr = FN(dot)(n, r, r, rev);
@@ -139,7 +151,9 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
             if (!(sigma > 0.0)) { status = ORC_BREAKDOWN; break; }
             const double alpha = rho / sigma;
             const T a = (T)alpha;
+            #pragma omp parallel for schedule(static)
             for (int32_t i = 0; i < n; ++i) x[i] = x[i] + a * p[i];
+            #pragma omp parallel for schedule(static)
             for (int32_t i = 0; i < n; ++i) r[i] = r[i] - a * q[i];
             k = k + 1;
             rr = FN(dot)(n, r, r, rev);
@@ -147,10 +161,12 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
             if (!fixed && sqrt(rr) <= tol) { status = ORC_CONVERGED; break; }
             if (rr == 0.0) { status = ORC_CONVERGED; break; }
             if (k == limit) break;
+            #pragma omp parallel for schedule(static)
             for (int32_t i = 0; i < n; ++i) q[i] = dinv[i] * r[i];   /* q holds z */
             const double rho_new = FN(dot)(n, r, q, rev);
             const double beta = rho_new / rho;
             const T bt = (T)beta;
+            #pragma omp parallel for schedule(static)
             for (int32_t i = 0; i < n; ++i) p[i] = q[i] + bt * p[i];
             rho = rho_new;
         }
@@ -172,6 +188,7 @@ int32_t FN(orc_pcg)(int32_t n, const int32_t *rowptr, const int32_t *colind,
 void FN(orc_grad_values)(int32_t n_rows, const int32_t *rowptr, const int32_t *colind,
                          const T *lambda, const T *x, T *grad, int32_t accumulate)
 {
+    #pragma omp parallel for schedule(static)
     for (int32_t i = 0; i < n_rows; ++i)
         for (int32_t t = rowptr[i]; t < rowptr[i + 1]; ++t) {
             const T g = -(lambda[i] * x[colind[t]]);
@@ -195,6 +212,7 @@ int32_t FN(orc_cg_adjoint)(int32_t n, const int32_t *rowptr, const int32_t *coli
     T *vT = (T *)malloc(sizeof(T) * (size_t)(nnz > 0 ? nnz : 1));
     if (!rpT || !ciT || !perm || !vT) { free(rpT); free(ciT); free(perm); free(vT); return -1; }
     orc_transpose_pattern(n, n, rowptr, colind, rpT, ciT, perm);
+    #pragma omp parallel for schedule(static)
     for (int32_t t = 0; t < nnz; ++t) vT[t] = vals[perm[t]];
     const int32_t rc = FN(orc_pcg)(n, rpT, ciT, vT, g, lambda, opt, res);
     free(rpT); free(ciT); free(perm); free(vT);
