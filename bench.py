@@ -377,15 +377,14 @@ def l2_stream_peak_gbs(dev) -> float:
     repeated), as the denominator of kernels whose working set stays in L2."""
     import torch
     buf = torch.ones(6 << 20, dtype=torch.float64, device=dev)     # 48 MB < 126 MB L2
-    out = torch.empty((), dtype=torch.float64, device=dev)
     for _ in range(5):
-        torch.sum(buf, out=out)
+        buf.sum()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = 50
     e0.record()
     for _ in range(reps):
-        torch.sum(buf, out=out)
+        buf.sum()
     e1.record()
     e1.synchronize()
     return buf.numel() * 8 * reps / (e0.elapsed_time(e1) / 1000.0) / 1e9

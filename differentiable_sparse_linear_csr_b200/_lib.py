@@ -12,7 +12,11 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
+# SLA_LIBRARY_VARIANT=debug_bounds selects the bounds-checking build
+# (libsla_debug_bounds.so); read once, when the library is first loaded.
+_VARIANT = os.environ.get("SLA_LIBRARY_VARIANT", "")
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         f"libsla{'_' + _VARIANT if _VARIANT else ''}.so")
 
 SLA_F64, SLA_F32 = 0, 1
 SLA_OK, SLA_ERR_INVALID, SLA_ERR_CUDA, SLA_ERR_OOM, SLA_ERR_TIMEOUT, SLA_ERR_UNSUPPORTED = range(6)
@@ -20,6 +24,7 @@ SLA_CONVERGED, SLA_NOT_CONVERGED, SLA_BREAKDOWN, SLA_NONFINITE, SLA_FIXED_DONE, 
 SLA_FLAG_VALIDATE, SLA_FLAG_SYMMETRIC, SLA_FLAG_BUILD_TRANSPOSE = 1, 2, 4
 SLA_STRATEGY_AUTO, SLA_STRATEGY_GRID, SLA_STRATEGY_BLOCK, SLA_STRATEGY_CLUSTER = 0, 1, 2, 3
 SLA_OP_SPMV, SLA_OP_CG, SLA_OP_ADJOINT, SLA_OP_GRAD = 0, 1, 2, 3
+SLA_GRAD_ACCUMULATE, SLA_GRAD_SHIFT_SHARED = 1, 2
 
 STATUS_NAMES = {0: "converged", 1: "not_converged", 2: "breakdown", 3: "nonfinite",
                 4: "fixed_done", 5: "timed_out"}
@@ -70,6 +75,7 @@ _SIGNATURES = {
     "sla_cg_solve": ([_P, _P, _P, _P, ctypes.POINTER(sla_cg_opts), sla_cg_info, _P, _SZ, _P], _I32),
     "sla_cg_adjoint": ([_P, _P, _P, _P, ctypes.POINTER(sla_cg_opts), sla_cg_info, _P, _SZ, _P], _I32),
     "sla_grad_values": ([_P, _P, _P, _P, _I32, _P], _I32),
+    "sla_matvec_grad_values": ([_P, _P, _P, _P, _I32, _P], _I32),
     "sla_transpose_workspace_bytes": ([_I32, _I32, _I64], _SZ),
     "sla_csr_transpose": ([_I32, _I32, _I64, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "sla_coo_workspace_bytes": ([_I32, _I32, _I64], _SZ),
@@ -84,6 +90,8 @@ _SIGNATURES = {
     "sla_edges_workspace_bytes": ([_P], _SZ),
     "sla_laplacian_grad_values": ([_P, _P, _P, _P, _I32, _P, _SZ, _P], _I32),
     "sla_laplacian_grad": ([_P, _P, _P, _P, _P, _I32, _P, _SZ, _P], _I32),
+    "sla_debug_bounds_report": ([ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(_I32), ctypes.POINTER(_I64),
+                                 _I32], _I32),
     "sla_last_error_string": ([], ctypes.c_char_p),
     "sla_version": ([], ctypes.c_char_p),
 }
@@ -141,6 +149,14 @@ def dtype_code(dtype: torch.dtype) -> int:
 # --------------------------------------------------------------------------
 # One function per C entry point, same names.
 # --------------------------------------------------------------------------
+
+def sla_debug_bounds_report(reset: bool = False) -> tuple[int, int, int]:
+    """(violations, first code, first index) of the bounds-checking build."""
+    v, c, i = ctypes.c_uint64(), _I32(), _I64()
+    _check("sla_debug_bounds_report", lib().sla_debug_bounds_report(ctypes.byref(v), ctypes.byref(c),
+                                                                    ctypes.byref(i), int(reset)))
+    return int(v.value), int(c.value), int(i.value)
+
 
 def sla_version() -> str:
     return lib().sla_version().decode()
@@ -218,6 +234,11 @@ def sla_grad_values(h, lam, x, grad, accumulate=0, stream=None) -> None:
                                                     _stream(stream)))
 
 
+def sla_matvec_grad_values(h, gy, x, grad, accumulate=0, stream=None) -> None:
+    _check("sla_matvec_grad_values", lib().sla_matvec_grad_values(h, _ptr(gy), _ptr(x), _ptr(grad),
+                                                                  int(accumulate), _stream(stream)))
+
+
 def sla_transpose_workspace_bytes(n_rows, n_cols, nnz) -> int:
     return int(lib().sla_transpose_workspace_bytes(n_rows, n_cols, nnz))
 
@@ -288,13 +309,13 @@ def sla_edges_workspace_bytes(e) -> int:
     return int(lib().sla_edges_workspace_bytes(e))
 
 
-def sla_laplacian_grad_values(e, G, dw, dshift, accumulate, ws, stream=None) -> None:
+def sla_laplacian_grad_values(e, G, dw, dshift, flags, ws, stream=None) -> None:
     _check("sla_laplacian_grad_values", lib().sla_laplacian_grad_values(
-        e, _ptr(G), _ptr(dw), _ptr(dshift), int(accumulate), _ptr(ws),
+        e, _ptr(G), _ptr(dw), _ptr(dshift), int(flags), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def sla_laplacian_grad(e, lam, x, dw, dshift, accumulate, ws, stream=None) -> None:
+def sla_laplacian_grad(e, lam, x, dw, dshift, flags, ws, stream=None) -> None:
     _check("sla_laplacian_grad", lib().sla_laplacian_grad(
-        e, _ptr(lam), _ptr(x), _ptr(dw), _ptr(dshift), int(accumulate), _ptr(ws),
+        e, _ptr(lam), _ptr(x), _ptr(dw), _ptr(dshift), int(flags), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))

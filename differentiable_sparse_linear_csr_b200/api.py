@@ -136,6 +136,15 @@ class CSR:
         L.sla_grad_values(self.handle, lm, xv, g, int(accumulate))
         return g
 
+    def matvec_grad_values(self, gy, x, out=None, accumulate=False) -> torch.Tensor:
+        """dL/dvalues[t] = gy[row t] * x[col t] on the pattern (for y = A x)."""
+        gv = self._vec(gy, self.n_rows)
+        xv = self._vec(x, self.n_cols)
+        g = out if out is not None else torch.empty(self.batch, self.nnz, dtype=self.dtype,
+                                                    device=self.device)
+        L.sla_matvec_grad_values(self.handle, gv, xv, g, int(accumulate))
+        return g
+
     # ---------------------------------------------------- autograd calls
     def matvec(self, values, x) -> torch.Tensor:
         """y = A x, differentiable in values and x."""
@@ -226,8 +235,7 @@ class _MatVec(torch.autograd.Function):
         if ctx.needs_input_grad[2]:
             gx = A.spmv(values, gy, transpose=True).reshape(x.shape)
         if ctx.needs_input_grad[1]:
-            # dy_i/dA_ij = x_j, i.e. the value-gradient kernel with lambda = -gy
-            gv = A.grad_values(-gy, x).reshape(values.shape)
+            gv = A.matvec_grad_values(gy, x).reshape(values.shape)   # dy_i/dA_ij = x_j
         return None, gv, gx
 
 
@@ -312,27 +320,29 @@ class EdgeLaplacian:
         L.sla_laplacian_assemble(self.plan, self._w(w), self._shift(shift), vals)
         return vals
 
-    def _grads(self, fn, args, dw, dshift, accumulate):
+    def _grads(self, fn, args, dw, dshift, accumulate, want_shift, shared_shift):
         A = self.A
         dw = dw if dw is not None else torch.empty(A.batch, self.n_edges, dtype=A.dtype, device=A.device)
+        if dshift is None and want_shift:
+            dshift = torch.empty(1 if shared_shift else A.batch, dtype=A.dtype, device=A.device)
         ws = _workspace(L.sla_edges_workspace_bytes(self.plan), A.device) if dshift is not None else None
-        fn(self.plan, *args, dw, dshift, int(accumulate), ws)
+        flags = (L.SLA_GRAD_ACCUMULATE if accumulate else 0) | \
+            (L.SLA_GRAD_SHIFT_SHARED if shared_shift else 0)
+        fn(self.plan, *args, dw, dshift, flags, ws)
         return dw, dshift
 
-    def grad_from_values(self, G, dw=None, dshift=None, accumulate=False, want_shift=True):
-        """(dL/dw [B, E], dL/dshift [B]) from G = dL/dvalues by the chain rule."""
-        A = self.A
-        if dshift is None and want_shift:
-            dshift = torch.empty(A.batch, dtype=A.dtype, device=A.device)
-        return self._grads(L.sla_laplacian_grad_values, (A._values(G),), dw, dshift, accumulate)
+    def grad_from_values(self, G, dw=None, dshift=None, accumulate=False, want_shift=True,
+                         shared_shift=False):
+        """(dL/dw [B, E], dL/dshift [B]) from G = dL/dvalues by the chain rule;
+        with shared_shift, dL/dshift [1] of one shift that serves every system."""
+        return self._grads(L.sla_laplacian_grad_values, (self.A._values(G),), dw, dshift, accumulate,
+                           want_shift, shared_shift)
 
-    def grad(self, lam, x, dw=None, dshift=None, accumulate=False, want_shift=True):
+    def grad(self, lam, x, dw=None, dshift=None, accumulate=False, want_shift=True, shared_shift=False):
         """The same for G = -lam x^T on the pattern, without forming G."""
         A = self.A
-        if dshift is None and want_shift:
-            dshift = torch.empty(A.batch, dtype=A.dtype, device=A.device)
         return self._grads(L.sla_laplacian_grad, (A._vec(lam, A.n_rows), A._vec(x, A.n_rows)),
-                           dw, dshift, accumulate)
+                           dw, dshift, accumulate, want_shift, shared_shift)
 
     # ---------------------------------------------------- autograd calls
     def assemble(self, w, shift=None) -> torch.Tensor:
@@ -358,10 +368,10 @@ class _Assemble(torch.autograd.Function):
     def backward(ctx, gv):
         E = ctx.E
         want_s = ctx.needs_input_grad[2]
-        dw, ds = E.grad_from_values(gv.contiguous(), want_shift=want_s)
+        shared = want_s and math.prod(ctx.shift_shape) == 1 and E.A.batch > 1
+        dw, ds = E.grad_from_values(gv.contiguous(), want_shift=want_s, shared_shift=shared)
         gw = dw.reshape(gv.shape[:-1] + (E.n_edges,)) if ctx.needs_input_grad[1] else None
-        gs = ds.reshape(ctx.shift_shape) if want_s and ds.numel() == math.prod(ctx.shift_shape) else \
-            (ds.sum().reshape(ctx.shift_shape) if want_s else None)
+        gs = ds.reshape(ctx.shift_shape) if want_s else None
         return None, gw, gs
 
 
@@ -388,11 +398,11 @@ class _EdgeSolve(torch.autograd.Function):
         want_s = ctx.needs_input_grad[2]
         gw = gs = None
         if ctx.needs_input_grad[1] or want_s:
-            dw, ds = E.grad(lam, x, want_shift=want_s)
+            shared = want_s and math.prod(ctx.shift_shape) == 1 and A.batch > 1
+            dw, ds = E.grad(lam, x, want_shift=want_s, shared_shift=shared)
             gw = dw.reshape(ctx.w_shape) if ctx.needs_input_grad[1] else None
             if want_s:
-                gs = ds.reshape(ctx.shift_shape) if ds.numel() == math.prod(ctx.shift_shape) else \
-                    ds.sum().reshape(ctx.shift_shape)
+                gs = ds.reshape(ctx.shift_shape)
         gb = lam.reshape(gx.shape) if ctx.needs_input_grad[3] else None
         return None, gw, gs, gb, None
 

@@ -39,7 +39,6 @@
 
 #include <algorithm>
 #include <climits>
-#include <mutex>
 #include <vector>
 
 #include "sla_rows.cuh"
@@ -75,6 +74,10 @@ struct CgArgs {
     const T *sell_vals;                     // [B][sell_nnz] values in that layout
     const SellRec<T> *sell_rec;             // or [B][sell_nnz] value-and-column records
     int64_t sell_nnz;
+    int sell_w;         // > 0: every slice of the sliced layout is sell_w entries wide
+    const int32_t *sell_perm;   // or null: the row at each position of the sliced layout
+    int ldmode;         // sliced-matrix load mode of the HBM solver (see sell_load)
+    int l2_prefetch;    // HBM solver: row waves of the matrix stream prefetched into L2 ahead
 };
 
 // ------------------------------------------------------------ helpers ----
@@ -270,19 +273,54 @@ __device__ void give_up(const CgArgs<T> &a) {
 }
 
 // ------------------------------------------------------- grid kernel ----
+constexpr int kMaxWaves = 128;   // row waves of one tile the L2 prefetch schedule covers
+
+// q = A p over rows [r0, r1) of the sliced layout with vectors in HBM, one row
+// a thread (rows r0 + tid, r0 + tid + NT, ...: "waves" of NT rows).  When
+// nwaves > 0, thread 0 keeps the matrix slots of the next D waves on their way
+// into L2 (bulk prefetch; wave_slot holds each wave's first slot).  Returns the
+// thread's partial p.q.
+template <int MODE, int NT, typename T>
+__device__ __forceinline__ double sell_tile_hbm(const CgArgs<T> &a, const T *svals, const T *pg, T *q_out,
+                                                int q_off, int r0, int r1, const int *wave_slot, int nwaves) {
+    const int tid = threadIdx.x, D = a.l2_prefetch;
+    auto prefetch = [&](int w) {
+        const int b0 = wave_slot[w], b1 = wave_slot[w + 1];
+        if (b1 > b0) {
+            prefetch_l2_bulk(svals + b0, (unsigned)((b1 - b0) * sizeof(T)));
+            prefetch_l2_bulk(a.sell_cols + b0, (unsigned)((b1 - b0) * sizeof(int32_t)));
+        }
+    };
+    if (nwaves > 0 && tid == 0)
+        for (int w = 0; w < D && w < nwaves; ++w) prefetch(w);
+    double acc = 0.0;
+    int w = 0;
+    for (int i = r0 + tid; i < r1; i += NT, ++w) {
+        if (nwaves > 0 && tid == 0 && w + D < nwaves) prefetch(w + D);
+        const T qi = sell_row<MODE>(a.sell_ptr, a.sell_cols, svals, pg, i, a.n, a.sell_nnz, a.sell_w);
+        const int row = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i), a.n, kBndLocal) : i;
+        q_out[row - q_off] = qi;
+        acc += (double)pg[row] * (double)qi;
+    }
+    return acc;
+}
+
 // Every block owns the tiles blockIdx.x + lt * gridDim.x (lt = 0, 1, ...) for
 // the whole solve and takes the decisions (breakdown, stop, alpha, beta) for
 // them itself from the shared partials; ONCHIP keeps x, r and M^-1 of its one
 // tile in shared memory and q in registers (RPT rows a thread), so only A and
-// p travel through L2/HBM each iteration.
-template <typename T, int LANES, bool ONCHIP, int RPT, int NT, bool SELL>
-__global__ void __launch_bounds__(NT, ONCHIP ? 1 : 2)
+// p travel through L2/HBM each iteration.  RQS (vectors otherwise in HBM, one
+// tile a block) keeps r and q of the tile in shared memory: for systems whose
+// three on-chip vectors do not fit, it saves the r and q passes over HBM.
+template <typename T, int LANES, bool ONCHIP, int RPT, int NT, bool SELL, bool RQS = false>
+__global__ void __launch_bounds__(NT, (ONCHIP || RQS) ? 1 : 2)
 cg_grid_kernel(CgArgs<T> a) {
+    static_assert(!(ONCHIP && RQS), "one on-chip layout at a time");
+    constexpr int LT = (ONCHIP || RQS) ? 1 : kMaxLocalTiles;   // tiles one block may own
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ double red[4 * 33];
-    __shared__ double l_rho[kMaxLocalTiles], l_nb[kMaxLocalTiles], l_rr[kMaxLocalTiles],
-        l_alpha[kMaxLocalTiles];
-    __shared__ int l_state[kMaxLocalTiles];
+    __shared__ double l_rho[LT], l_nb[LT], l_rr[LT], l_alpha[LT];
+    __shared__ int l_state[LT];
     __shared__ int flag;
     __shared__ unsigned active;
     constexpr int NSUB = NT / LANES;
@@ -303,8 +341,28 @@ cg_grid_kernel(CgArgs<T> a) {
     T *xs_ = reinterpret_cast<T *>(smem_raw);     // ONCHIP: [tile_rows] each
     T *rs_ = xs_ + (ONCHIP ? a.tile_rows : 0);
     T *ds_ = rs_ + (ONCHIP ? a.tile_rows : 0);
+    T *rq_ = reinterpret_cast<T *>(smem_raw);     // RQS: r [tile_rows], then q [tile_rows]
+    T *qq_ = rq_ + (RQS ? a.tile_rows : 0);
+    __shared__ int wave_slot[(SELL && !ONCHIP) ? kMaxWaves + 1 : 1];
+    int nwaves = 0;   // > 0: the SpMV prefetches its tile's matrix stream into L2
 
     if (blockIdx.x == 0 && tid == 0) a.sync[3] = (unsigned)a.B;
+    if constexpr (SELL && !ONCHIP) {
+        if (a.l2_prefetch > 0 && nlt == 1 && a.sell_rec == nullptr) {
+            const int tt = blockIdx.x % a.ntiles;
+            const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
+            const int nw = (r1 - r0 + NT - 1) / NT;
+            if (nw <= kMaxWaves) {
+                // wave w covers rows [r0 + w NT, min(r1, r0 + (w+1) NT)): its slots start at
+                // the slice holding its first row; the table ends at the slice after r1 - 1
+                for (int w = tid; w <= nw; w += NT) {
+                    const int sl = w < nw ? (r0 + w * NT) / kSellRows : (r1 + kSellRows - 1) / kSellRows;
+                    wave_slot[w] = __ldg(a.sell_ptr + sl);
+                }
+                nwaves = nw;
+            }
+        }
+    }
 
     // ---- init: r = b - A x0 (or b), z = M^-1 r, p = z; partials of b.b, r.z, r.r
     for (int lt = 0; lt < nlt; ++lt) {
@@ -316,7 +374,7 @@ cg_grid_kernel(CgArgs<T> a) {
         T *xg = a.x + (int64_t)s * n, *pg = a.p + (int64_t)s * n, *qg = a.q + (int64_t)s * n;
         if (a.x0_given) {
             for (int i = r0 + sub; i < r1; i += NSUB) {
-                const T v = row_dot<T, LANES>(a.rowptr, a.colind, vs, xg, i, lane);
+                const T v = row_dot<T, LANES>(a.rowptr, a.colind, vs, xg, i, lane, n, a.nnz);
                 if (lane == 0) qg[i] = v;
             }
             __syncthreads();
@@ -329,7 +387,7 @@ cg_grid_kernel(CgArgs<T> a) {
             T di = T(1);
             if (a.precond) {
                 const int dp = __ldg(a.diagpos + i);
-                const T dv = dp >= 0 ? __ldg(vs + dp) : T(0);
+                const T dv = dp >= 0 ? __ldg(vs + SLA_IDX(dp, a.nnz, kBndDiag)) : T(0);
                 if (!(dv > T(0))) acc[3] += 1.0;
                 di = T(1) / dv;
             }
@@ -341,7 +399,8 @@ cg_grid_kernel(CgArgs<T> a) {
                 ds_[i - r0] = di;
             } else {
                 if (!a.x0_given) xg[i] = T(0);
-                a.r[(int64_t)s * n + i] = ri;
+                if constexpr (RQS) rq_[i - r0] = ri;
+                else a.r[(int64_t)s * n + i] = ri;
                 a.d[(int64_t)s * n + i] = di;
             }
             acc[0] += (double)bi * (double)bi;
@@ -427,7 +486,7 @@ cg_grid_kernel(CgArgs<T> a) {
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
                         if (i < r1) {
-                            const T qi = sell_row_rec<false>(a.sell_ptr, rec, pg, i);
+                            const T qi = sell_row_rec<false>(a.sell_ptr, rec, pg, i, n, a.sell_nnz);
                             qreg[j] = qi;
                             acc[0] += (double)pg[i] * (double)qi;
                         }
@@ -438,7 +497,7 @@ cg_grid_kernel(CgArgs<T> a) {
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
                         if (i < r1) {
-                            const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i);
+                            const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i, n, a.sell_nnz, a.sell_w);
                             qreg[j] = qi;
                             acc[0] += (double)pg[i] * (double)qi;
                         }
@@ -449,34 +508,38 @@ cg_grid_kernel(CgArgs<T> a) {
                 for (int j = 0; j < RPT; ++j) {
                     const int i = r0 + tid + j * NT;
                     if (i < r1) {
-                        const T qi = row_dot<T, 1>(a.rowptr, a.colind, vs, pg, i, 0);
+                        const T qi = row_dot<T, 1>(a.rowptr, a.colind, vs, pg, i, 0, n, a.nnz);
                         qreg[j] = qi;
                         acc[0] += (double)pg[i] * (double)qi;
                     }
                 }
             } else if constexpr (SELL) {
-                T *qg = a.q + (int64_t)s * n;
+                T *qg = RQS ? qq_ : a.q + (int64_t)s * n;   // q of row i at qg[i - qoff]
+                const int qoff = RQS ? r0 : 0;
                 if (a.sell_rec) {
                     const SellRec<T> *rec = a.sell_rec + (int64_t)s * a.sell_nnz;
                     for (int i = r0 + tid; i < r1; i += NT) {
-                        const T qi = sell_row_rec<true>(a.sell_ptr, rec, pg, i);
-                        qg[i] = qi;
-                        acc[0] += (double)pg[i] * (double)qi;
+                        const T qi = sell_row_rec<true>(a.sell_ptr, rec, pg, i, n, a.sell_nnz);
+                        const int row = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i), n, kBndLocal) : i;
+                        qg[row - qoff] = qi;
+                        acc[0] += (double)pg[row] * (double)qi;
                     }
                 } else {
                     const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
-                    for (int i = r0 + tid; i < r1; i += NT) {
-                        const T qi = sell_row<true>(a.sell_ptr, a.sell_cols, svals, pg, i);
-                        qg[i] = qi;
-                        acc[0] += (double)pg[i] * (double)qi;
+                    switch (a.ldmode) {
+                        case 0: acc[0] = sell_tile_hbm<0, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
+                        case 2: acc[0] = sell_tile_hbm<2, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
+                        case 3: acc[0] = sell_tile_hbm<3, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
+                        default: acc[0] = sell_tile_hbm<1, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
                     }
                 }
             } else {
-                T *qg = a.q + (int64_t)s * n;
+                T *qg = RQS ? qq_ : a.q + (int64_t)s * n;   // q of row i at qg[i - qoff]
+                const int qoff = RQS ? r0 : 0;
                 for (int i = r0 + sub; i < r1; i += NSUB) {
-                    const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, pg, i, lane);
+                    const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, pg, i, lane, n, a.nnz);
                     if (lane == 0) {
-                        qg[i] = qi;
+                        qg[i - qoff] = qi;
                         acc[0] += (double)pg[i] * (double)qi;
                     }
                 }
@@ -522,12 +585,14 @@ cg_grid_kernel(CgArgs<T> a) {
                     }
                 }
             } else {
-                T *rg = a.r + (int64_t)s * n;
-                const T *qg = a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                // r and q of row i at rg[i - off], qg[i - off]
+                T *rg = RQS ? rq_ : a.r + (int64_t)s * n;
+                const T *qg = RQS ? qq_ : a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                const int off = RQS ? r0 : 0;
 #pragma unroll 4
                 for (int i = r0 + tid; i < r1; i += NT) {
-                    const T ri = rg[i] - al * qg[i];
-                    rg[i] = ri;
+                    const T ri = rg[i - off] - al * qg[i - off];
+                    rg[i - off] = ri;
                     const T zi = dg[i] * ri;
                     acc[0] += (double)ri * (double)zi;
                     acc[1] += (double)ri * (double)ri;
@@ -592,9 +657,10 @@ cg_grid_kernel(CgArgs<T> a) {
                         if (i < r1) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pg[i];
                     }
                 } else {
-                    const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                    const T *rg = RQS ? rq_ : a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
+                    const int off = RQS ? r0 : 0;
 #pragma unroll 4
-                    for (int i = r0 + tid; i < r1; i += NT) pg[i] = dg[i] * rg[i] + bt * pg[i];
+                    for (int i = r0 + tid; i < r1; i += NT) pg[i] = dg[i] * rg[i - off] + bt * pg[i];
                 }
             }
             __syncthreads();
@@ -668,7 +734,7 @@ cg_grid2_kernel(CgArgs<T> a) {
 #pragma unroll
             for (int j = 0; j < RPT; ++j) {
                 const int i = r0 + tid + j * NT;
-                if (i < r1) qreg[j] = row_dot<T, 1>(a.rowptr, a.colind, a.vals, a.x, i, 0);
+                if (i < r1) qreg[j] = row_dot<T, 1>(a.rowptr, a.colind, a.vals, a.x, i, 0, a.n, a.nnz);
             }
         }
 #pragma unroll
@@ -681,7 +747,7 @@ cg_grid2_kernel(CgArgs<T> a) {
                 T di = T(1);
                 if (a.precond) {
                     const int dp = __ldg(a.diagpos + i);
-                    const T dv = dp >= 0 ? __ldg(a.vals + dp) : T(0);
+                    const T dv = dp >= 0 ? __ldg(a.vals + SLA_IDX(dp, a.nnz, kBndDiag)) : T(0);
                     if (!(dv > T(0))) acc[3] += 1.0;
                     di = T(1) / dv;
                 }
@@ -735,7 +801,7 @@ cg_grid2_kernel(CgArgs<T> a) {
         for (int j = 0; j < RPT; ++j) {
             const int i = r0 + tid + j * NT;
             if (i < r1) {
-                const T qi = sell_row_dir<T>(a.sell_ptr, a.sell_cols, svals, zg, pprev, bt, i);
+                const T qi = sell_row_dir<T>(a.sell_ptr, a.sell_cols, svals, zg, pprev, bt, i, a.n, a.sell_nnz, a.sell_w);
                 qreg[j] = qi;
                 T pi;
                 if constexpr (sizeof(T) == 8) pi = __fma_rn(bt, pprev[i], __dmul_rn(ds[i - r0], rs[i - r0]));
@@ -835,8 +901,8 @@ cg_block_kernel(CgArgs<T> a) {
             __syncthreads();
         }
         auto spmv_row = [&](const T *v, int i) -> T {
-            if constexpr (MRES) return row_dot_shared<T, LANES>(rp_s, cols_s, vals_s, v, i, lane);
-            else return row_dot<T, LANES>(a.rowptr, a.colind, vs, v, i, lane);
+            if constexpr (MRES) return row_dot_shared<T, LANES>(rp_s, cols_s, vals_s, v, i, lane, n, a.nnz);
+            else return row_dot<T, LANES>(a.rowptr, a.colind, vs, v, i, lane, n, a.nnz);
         };
         if (a.x0_given) {
             for (int i = tid; i < n; i += kCgThreads) xs[i] = xg[i];
@@ -860,7 +926,7 @@ cg_block_kernel(CgArgs<T> a) {
             T di = T(1);
             if (a.precond) {
                 const int dp = __ldg(a.diagpos + i);
-                const T dv = dp >= 0 ? __ldg(vs + dp) : T(0);
+                const T dv = dp >= 0 ? __ldg(vs + SLA_IDX(dp, a.nnz, kBndDiag)) : T(0);
                 if (!(dv > T(0))) bad += 1.0;
                 di = T(1) / dv;
             }
@@ -971,7 +1037,8 @@ struct VecLoad {
 
 template <typename T, int BW>
 __device__ __forceinline__ void il_row(const int32_t *__restrict__ sptr, const int32_t *__restrict__ cols,
-                                       const T *__restrict__ sv, const T *v, int i, T (&q)[BW]) {
+                                       const T *__restrict__ sv, const T *v, int i, T (&q)[BW],
+                                       int ncols, int64_t nslots) {
     const int sl = i / kSellRows;
     const int b0 = __ldg(sptr + sl);
     const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
@@ -979,8 +1046,8 @@ __device__ __forceinline__ void il_row(const int32_t *__restrict__ sptr, const i
 #pragma unroll
     for (int s = 0; s < BW; ++s) q[s] = T(0);
     for (int k = 0; k < w; ++k) {
-        const int t = base + k * kSellRows;
-        const int c = sell_load<true>(cols + t);
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        const int c = SLA_IDX(sell_load<true>(cols + t), ncols, kBndColumn);
         T av[BW], pv[BW];
         VecLoad<T, BW>::ld(sv + (int64_t)t * BW, av);
         VecLoad<T, BW>::ld(v + (int64_t)c * BW, pv);
@@ -1021,8 +1088,8 @@ cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, 
         for (int j = 0; j < 4 * BW; ++j) acc[j] = 0.0;
         for (int i = r0 + tid; i < r1; i += NT) {
             T qx[BW];
-            if (a.x0_given) il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, xi, i, qx);
-            const int dp = a.precond ? __ldg(a.diagpos + i) : -1;
+            if (a.x0_given) il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, xi, i, qx, a.n, a.sell_nnz);
+            const int dp = a.precond ? SLA_IDX(__ldg(a.diagpos + i), a.nnz, kBndDiag) : -1;
 #pragma unroll
             for (int s = 0; s < BW; ++s) {
                 const int64_t o = (int64_t)i * BW + s;
@@ -1095,7 +1162,7 @@ cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, 
             for (int s = 0; s < BW; ++s) acc[s] = 0.0;
             for (int i = r0 + tid; i < r1; i += NT) {
                 T qv[BW], pv[BW];
-                il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, p, i, qv);
+                il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, p, i, qv, a.n, a.sell_nnz);
                 VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
                 VecLoad<T, BW>::st(q + (int64_t)i * BW, qv);
 #pragma unroll
@@ -1302,7 +1369,10 @@ cg_segment_kernel(CgArgs<T> a, const int32_t *__restrict__ seg, const int32_t *_
         auto spmv_row = [&](const T *v, int li) -> T {
             const int t0 = __ldg(a.rowptr + o + li), t1 = __ldg(a.rowptr + o + li + 1);
             T acc = T(0);
-            for (int t = t0 + lane; t < t1; t += LANES) acc += __ldg(a.vals + t) * v[__ldg(a.colind + t) - o];
+            for (int t = t0 + lane; t < t1; t += LANES) {
+                const int tt = SLA_IDX(t, a.nnz, kBndEntry);
+                acc += __ldg(a.vals + tt) * v[SLA_IDX(__ldg(a.colind + tt) - o, m, kBndLocal)];
+            }
             if constexpr (LANES > 1) {
                 const unsigned mk = subwarp_mask<LANES>();
 #pragma unroll
@@ -1334,7 +1404,7 @@ cg_segment_kernel(CgArgs<T> a, const int32_t *__restrict__ seg, const int32_t *_
             T di = T(1);
             if (a.precond) {
                 const int dp = __ldg(a.diagpos + o + i);
-                const T dv = dp >= 0 ? __ldg(a.vals + dp) : T(0);
+                const T dv = dp >= 0 ? __ldg(a.vals + SLA_IDX(dp, a.nnz, kBndDiag)) : T(0);
                 if (!(dv > T(0))) bad += 1.0;
                 di = T(1) / dv;
             }
@@ -1516,8 +1586,9 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
     const int t0 = m > 0 ? __ldg(a.rowptr + r0) : 0, t1 = m > 0 ? __ldg(a.rowptr + r1) : 0;
     for (int i = tid; i <= m; i += NT) rp_s[i] = m > 0 ? __ldg(a.rowptr + r0 + i) - t0 : 0;
     for (int t = t0 + tid; t < t1; t += NT) {
-        c_s[t - t0] = __ldg(a.colind + t);
-        v_s[t - t0] = __ldg(vs + t);
+        const int lt = SLA_IDX(t - t0, nnz_cap, kBndLocal);
+        c_s[lt] = __ldg(a.colind + SLA_IDX(t, a.nnz, kBndEntry));
+        v_s[lt] = __ldg(vs + SLA_IDX(t, a.nnz, kBndEntry));
     }
     __syncthreads();
 
@@ -1556,7 +1627,7 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
             T ax = T(0);
             for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) {
                 if (c_s[t] == i) dv = v_s[t];
-                if (a.x0_given) ax += v_s[t] * xg[c_s[t]];
+                if (a.x0_given) ax += v_s[t] * xg[SLA_IDX(c_s[t], n, kBndColumn)];
             }
             if (a.x0_given) {
                 xi = xg[i];
@@ -1599,8 +1670,8 @@ cg_cluster_kernel(CgArgs<T> a, int rows_cta, int nnz_cap) {
         for (int li = tid; li < m; li += NT) {
             T qi = T(0);
             for (int t = rp_s[li]; t < rp_s[li + 1]; ++t) {
-                const int j = c_s[t];
-                const int o = j / rows_cta, lj = j - o * rows_cta;
+                const int j = SLA_IDX(c_s[t], n, kBndColumn);
+                const int o = SLA_IDX(j / rows_cta, CS, kBndLocal), lj = j - o * rows_cta;
                 qi += v_s[t] * direction(db[o][lj], rb[o][lj], pb[prev][o][lj], bt);
             }
             q_s[li] = qi;
@@ -1671,6 +1742,10 @@ template <typename T, int RPT, bool SELL>
 static const void *onchip_fn() {
     return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads, SELL>);
 }
+template <typename T, bool SELL>
+static const void *rqs_fn() {
+    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, false, 1, kOnchipThreads, SELL, true>);
+}
 template <typename T, int RPT>
 static const void *grid2_fn() {
     return reinterpret_cast<const void *>(&cg_grid2_kernel<T, RPT, kOnchipThreads>);
@@ -1729,8 +1804,14 @@ static const void *pick_il(sla_dtype dt, int B) {
                   : reinterpret_cast<const void *>(&cg_grid_il_kernel<float, 4>);
 }
 
+static const void *pick_rqs(sla_dtype dt, bool sell) {
+    if (dt == SLA_F64) return sell ? rqs_fn<double, true>() : rqs_fn<double, false>();
+    return sell ? rqs_fn<float, true>() : rqs_fn<float, false>();
+}
+
 static const void *pick_grid(const Csr *h, bool sell) {
     if (h->onchip) return pick_onchip(h->dtype, h->onchip_rpt, sell);
+    if (h->rqs) return pick_rqs(h->dtype, sell);
     if (sell) return h->dtype == SLA_F64 ? grid_sell_fn<double>() : grid_sell_fn<float>();
     return pick_fn(true, h->dtype, h->lanes);
 }
@@ -1791,8 +1872,9 @@ sla_status cg_configure(Csr *h) {
     // On-chip variant: one 1024-thread block per SM, x, r, M^-1 of the block's
     // rows in shared memory, at most 16 rows a thread.
     h->onchip = false;
+    // SLA_GRID_ONCHIP=0: vectors in HBM; =2: only the r-and-q variant below
     const char *oc = getenv("SLA_GRID_ONCHIP");
-    if (h->lanes == 1 && n > 0 && !(oc && oc[0] == '0')) {
+    if (h->lanes == 1 && n > 0 && !(oc && (oc[0] == '0' || oc[0] == '2'))) {
         int32_t tr = 0, nt = 0;
         layout(h, h->num_sms, &tr, &nt);
         const int rpt = (tr + kOnchipThreads - 1) / kOnchipThreads;
@@ -1831,7 +1913,35 @@ sla_status cg_configure(Csr *h) {
             }
         }
     }
-    if (!h->onchip) {
+    // Vectors in HBM except r and q, which stay in shared memory: one 1024-thread
+    // block per SM whose tile's r and q fit (systems too large for the on-chip
+    // variant's three vectors, e.g. 2 M fp64 rows).  SLA_GRID_RQS=0 turns it off.
+    h->rqs = false;
+    const char *rq = getenv("SLA_GRID_RQS");
+    if (!h->onchip && h->lanes == 1 && n > 0 && !(oc && oc[0] == '0') && !(rq && rq[0] == '0')) {
+        int32_t tr = 0, nt = 0;
+        layout(h, h->num_sms, &tr, &nt);
+        const size_t smem = 2 * (size_t)tr * ts;
+        if ((int64_t)h->batch * nt <= h->num_sms && smem + 4096 <= (size_t)optin) {
+            for (int sv = 0; sv < 2; ++sv)
+                SLA_CHECK_CUDA(cudaFuncSetAttribute(pick_rqs(h->dtype, sv != 0),
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    optin - 4096));
+            int per_sm = 0;
+            SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, pick_rqs(h->dtype, true), kOnchipThreads, smem));
+            if (per_sm >= 1) {
+                h->rqs = true;
+                h->grid_smem = smem;
+                h->grid_threads = kOnchipThreads;
+                h->grid_blocks = h->num_sms;
+                h->tile_rows = tr;
+                h->ntiles = nt;
+                h->il_blocks = 0;
+            }
+        }
+    }
+    if (!h->onchip && !h->rqs) {
         int per_sm = 0;
         SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
             &per_sm, pick_fn(true, h->dtype, h->lanes), kCgThreads, 0));
@@ -2046,6 +2156,10 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
     a.timeout_ns = o->wait_timeout_ns > 0 ? o->wait_timeout_ns : kDefaultTimeoutNs;
     a.tile_rows = h->tile_rows;
     a.ntiles = h->ntiles;
+    a.ldmode = 1;
+    if (const char *e = getenv("SLA_LDMODE")) a.ldmode = atoi(e);
+    a.l2_prefetch = 0;
+    if (const char *e = getenv("SLA_L2_PREFETCH")) a.l2_prefetch = atoi(e);
     if (h->dep_lo != nullptr && pattern_is_forward_or_sym(h, rowptr)) {
         a.dep_lo = h->dep_lo;
         a.dep_hi = h->dep_hi;
@@ -2136,6 +2250,8 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             a.sell_ptr = h->sell_ptr;
             a.sell_cols = h->sell_cols;
             a.sell_nnz = h->sell_nnz;
+            a.sell_w = h->sell_w;
+            a.sell_perm = h->sell_perm;
             const char *pk = getenv("SLA_SELL_PACK");
             const bool pack = pk && pk[0] == '1' && !(h->grid2 && a.B == 1);
             if (pack) {
@@ -2235,6 +2351,7 @@ extern "C" size_t sla_workspace_bytes(sla_csr_t hh, int32_t op) {
 extern "C" sla_status sla_cg_solve(sla_csr_t hh, const void *vals, const void *b, void *x,
                                    const sla_cg_opts *opts, sla_cg_info info, void *ws,
                                    size_t ws_bytes, void *stream) {
+    SLA_RANGE("sla_cg_solve");
     clear_error();
     return cg_entry(reinterpret_cast<Csr *>(hh), vals, b, x, opts, info, ws, ws_bytes, stream, false);
 }
@@ -2242,6 +2359,7 @@ extern "C" sla_status sla_cg_solve(sla_csr_t hh, const void *vals, const void *b
 extern "C" sla_status sla_cg_adjoint(sla_csr_t hh, const void *vals, const void *g, void *lambda,
                                      const sla_cg_opts *opts, sla_cg_info info, void *ws,
                                      size_t ws_bytes, void *stream) {
+    SLA_RANGE("sla_cg_adjoint");
     clear_error();
     return cg_entry(reinterpret_cast<Csr *>(hh), vals, g, lambda, opts, info, ws, ws_bytes, stream,
                     true);
@@ -2263,28 +2381,20 @@ namespace sla {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kNoAllocMaxDevices = 64;
-static void *g_noalloc_ptr[kNoAllocMaxDevices];
-static std::once_flag g_noalloc_once[kNoAllocMaxDevices];
-static cudaError_t g_noalloc_err[kNoAllocMaxDevices];
-
 // Host code sees g_noalloc_scratch only as a host-side stand-in; the device
-// address comes from cudaGetSymbolAddress, once per device, with that device
-// current.
-static sla_status noalloc_scratch(int device, void **out) {
-    if (device < 0 || device >= kNoAllocMaxDevices) {
-        set_error("sla_cg_solve_noalloc: device %d beyond the supported %d", device, kNoAllocMaxDevices);
-        return SLA_ERR_UNSUPPORTED;
-    }
-    std::call_once(g_noalloc_once[device], [device] {
-        g_noalloc_err[device] = cudaGetSymbolAddress(&g_noalloc_ptr[device], g_noalloc_scratch);
-    });
-    if (g_noalloc_err[device] != cudaSuccess || g_noalloc_ptr[device] == nullptr) {
-        set_error("sla_cg_solve_noalloc: cudaGetSymbolAddress failed: %s",
-                  cudaGetErrorString(g_noalloc_err[device]));
+// address comes from cudaGetSymbolAddress with the caller's context current.
+// It is looked up on every call (a host-side table lookup once the module is
+// loaded): a cached address would go stale when the caller switches to another
+// context of the same device or resets the device, because the library's
+// module, and with it the array, is then loaded again at another address.
+static sla_status noalloc_scratch(void **out) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+        set_error("sla_cg_solve_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
         return SLA_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[device];
+    *out = p;
     return SLA_OK;
 }
 
@@ -2347,6 +2457,7 @@ extern "C" sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t
                                            const void *vals, const void *b, void *x,
                                            const sla_cg_opts *opts, sla_cg_info info,
                                            void *stream) {
+    SLA_RANGE("sla_cg_solve_noalloc");
     clear_error();
     SLA_REQUIRE(n >= 0 && nnz >= 0 && nnz <= 0x7fffffff, "sla_cg_solve_noalloc: bad sizes n=%d nnz=%lld",
                 n, (long long)nnz);
@@ -2397,7 +2508,7 @@ extern "C" sla_status sla_cg_solve_noalloc(int32_t n, int64_t nnz, const int32_t
                 "built-in limit is %zu bytes (use sla_cg_solve with a caller workspace)",
                 batch, n, need, kNoAllocScratchBytes);
     void *scratch = nullptr;
-    st = noalloc_scratch(h.device, &scratch);
+    st = noalloc_scratch(&scratch);
     if (st != SLA_OK) return st;
     if (dtype == SLA_F64)
         return noalloc_launch<double>(h, (const double *)vals, (const double *)b, (double *)x, opts,

@@ -4,11 +4,13 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <cstdarg>
 #include <cstdio>
 #include <string>
+#include <type_traits>
 
 #include "../../include/sla.h"
 
@@ -47,6 +49,17 @@ void clear_error();
     } while (0)
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Names a C entry point in profiler timelines (an NVTX range around the call,
+// which encloses the kernels it enqueues); without a profiler attached the
+// push and pop do nothing.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
+#define SLA_RANGE(name) ::sla::Range sla_range_(name)
 
 inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
@@ -95,6 +108,7 @@ struct Csr {
     bool onchip = false;               // grid solver keeps x, r, M^-1 in shared memory
     int32_t onchip_rpt = 0;            // rows a thread in the on-chip grid solver
     bool grid2 = false;                // single system, on chip, sliced: two barriers an iteration
+    bool rqs = false;                  // grid solver keeps r and q in shared memory (x, M^-1 in HBM)
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
@@ -120,6 +134,9 @@ struct Csr {
     // together (padded to the slice's longest row).
     bool has_sell = false;
     int64_t sell_nnz = 0;              // stored entries including padding
+    int32_t sell_w = 0;                // > 0: every slice padded to this width (no offsets needed)
+    int32_t *sell_perm = nullptr;      // owned [n_rows] or null: row at each position (rows of each
+                                       // 32-row window ordered by decreasing length)
     int32_t *sell_ptr = nullptr;       // owned [n_slices + 1]: first entry of each slice
     int32_t *sell_cols = nullptr;      // owned [sell_nnz]: column (own row for padding)
     int32_t *sell_map = nullptr;       // owned [sell_nnz]: CSR position, -1 for padding
@@ -150,7 +167,10 @@ sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws
 
 // Sliced layout (built at handle creation for short-row square patterns).
 constexpr int kSellRows = 8;
-sla_status build_sell(Csr *h, cudaStream_t s);
+constexpr int kSellSortWindow = 32;   // rows sorted by length together (one warp's rows)
+// sort_ok: the solver that uses this layout keeps q by row index (vectors in
+// HBM or r and q in shared memory), so rows may be permuted within windows.
+sla_status build_sell(Csr *h, bool sort_ok, cudaStream_t s);
 sla_status cg_tile_deps(Csr *h, cudaStream_t s);   // in sla_cg.cu
 // vals_sell[b][slot] = vals[b][sell_map[slot]] (0 for padding), every system.
 sla_status sell_values(const Csr *h, const void *vals, void *vals_sell, cudaStream_t s);
@@ -260,5 +280,62 @@ __device__ __forceinline__ bool grid_barrier(unsigned *sync, unsigned nblocks,
     __syncthreads();
     return *flag_smem != 0;
 }
+
+// ------------------------------------------------- bounds-checking build ----
+// With SLA_DEBUG_BOUNDS=1 (the library's debug_bounds variant) every index the
+// kernels take from the pattern (a column gathered from a vector, a CSR or
+// sliced-layout entry, a diagonal position, an edge's entry) and every
+// shared-memory or cluster-rank index derived from it is checked against its
+// range before use.  A bad index is recorded (a count, and the smallest
+// (code, index) pair) and replaced by 0, so the access stays in bounds and
+// nothing traps; sla_debug_bounds_report reads the record.  Without the flag
+// SLA_IDX is the index itself and no code is added.
+enum {
+    kBndColumn = 1,   // gathered column >= vector length
+    kBndEntry = 2,    // entry position outside the value / column arrays
+    kBndDiag = 3,     // diagonal position outside the entries
+    kBndLocal = 4,    // shared-memory index or cluster rank out of range
+    kBndEdge = 5      // edge endpoint or edge-to-entry slot out of range
+};
+
+#ifndef SLA_DEBUG_BOUNDS
+#define SLA_DEBUG_BOUNDS 0
+#endif
+
+#if SLA_DEBUG_BOUNDS
+// One record per translation unit (device variables of a file without
+// relocatable device code are the file's own); each registers its reader.
+namespace {
+__device__ unsigned long long dbg_count = 0;
+__device__ unsigned long long dbg_first = ~0ull;
+}  // namespace
+
+__device__ __forceinline__ long long dbg_index(long long i, long long n, int code) {
+    if ((unsigned long long)i < (unsigned long long)n) return i;
+    atomicAdd(&dbg_count, 1ull);
+    atomicMin(&dbg_first, ((unsigned long long)code << 56) | ((unsigned long long)i & ((1ull << 56) - 1)));
+    return 0;
+}
+#define SLA_IDX(i, n, code) \
+    ((std::decay_t<decltype(i)>)::sla::dbg_index((long long)(i), (long long)(n), (code)))
+
+using DbgReader = cudaError_t (*)(unsigned long long *count, unsigned long long *first, bool reset);
+int dbg_register(DbgReader f);   // sla_handle.cu
+namespace {
+cudaError_t dbg_read(unsigned long long *count, unsigned long long *first, bool reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(count, dbg_count, sizeof(unsigned long long));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(first, dbg_first, sizeof(unsigned long long));
+    if (e == cudaSuccess && reset) {
+        const unsigned long long zero = 0, none = ~0ull;
+        e = cudaMemcpyToSymbol(dbg_count, &zero, sizeof zero);
+        if (e == cudaSuccess) e = cudaMemcpyToSymbol(dbg_first, &none, sizeof none);
+    }
+    return e;
+}
+[[maybe_unused]] const int dbg_registered = dbg_register(&dbg_read);
+}  // namespace
+#else
+#define SLA_IDX(i, n, code) (i)
+#endif
 
 }  // namespace sla

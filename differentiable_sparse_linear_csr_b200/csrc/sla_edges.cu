@@ -117,7 +117,7 @@ assemble_kernel(int n, int64_t nnz, int B, int64_t E, const int32_t *__restrict_
     for (int t = t0; t < t1; ++t) {
         const int e = __ldg(emap + t);
         if (e >= 0) {
-            const T we = __ldg(wb + e);
+            const T we = __ldg(wb + SLA_IDX(e, E, kBndEdge));
             vb[t] = -we;
             d = d + we;
         } else if (__ldg(colind + t) == i) {
@@ -147,14 +147,14 @@ edge_grad_kernel(int n, int64_t nnz, int64_t E, const int32_t *__restrict__ ei,
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     const int b = blockIdx.y;
-    const int i = __ldg(ei + e), j = __ldg(ej + e);
+    const int i = SLA_IDX(__ldg(ei + e), n, kBndEdge), j = SLA_IDX(__ldg(ej + e), n, kBndEdge);
     T gii, gjj, gij, gji;
     if constexpr (FROM_G) {
         const T *gb = G + (int64_t)b * nnz;
-        gii = __ldg(gb + __ldg(diagpos + i));
-        gjj = __ldg(gb + __ldg(diagpos + j));
-        gij = __ldg(gb + __ldg(sij + e));
-        gji = __ldg(gb + __ldg(sji + e));
+        gii = __ldg(gb + SLA_IDX(__ldg(diagpos + i), nnz, kBndDiag));
+        gjj = __ldg(gb + SLA_IDX(__ldg(diagpos + j), nnz, kBndDiag));
+        gij = __ldg(gb + SLA_IDX(__ldg(sij + e), nnz, kBndEdge));
+        gji = __ldg(gb + SLA_IDX(__ldg(sji + e), nnz, kBndEdge));
     } else {
         const T *lb = lam + (int64_t)b * n, *xb = x + (int64_t)b * n;
         const T li = __ldg(lb + i), lj = __ldg(lb + j), xi = __ldg(xb + i), xj = __ldg(xb + j);
@@ -180,7 +180,7 @@ diag_partial_kernel(int n, int64_t nnz, int ntiles, const int32_t *__restrict__ 
     double s = 0.0;
     for (int i = r0 + threadIdx.x; i < r1; i += kEdgeThreads) {
         if constexpr (FROM_G) {
-            s += (double)__ldg(G + (int64_t)b * nnz + __ldg(diagpos + i));
+            s += (double)__ldg(G + (int64_t)b * nnz + SLA_IDX(__ldg(diagpos + i), nnz, kBndDiag));
         } else {
             const int64_t o = (int64_t)b * n + i;
             s += (double)neg_prod(__ldg(lam + o), __ldg(x + o));
@@ -190,14 +190,16 @@ diag_partial_kernel(int n, int64_t nnz, int ntiles, const int32_t *__restrict__ 
     if (threadIdx.x == 0) part[(int64_t)b * ntiles + blockIdx.x] = s;
 }
 
+// dshift[b] = the sum of block b's `count` partials (a fixed tree); with one
+// block over all B * ntiles partials this is the shared shift's gradient.
 template <typename T>
 __global__ void __launch_bounds__(kEdgeThreads)
-diag_finish_kernel(int ntiles, const double *__restrict__ part, T *__restrict__ dshift,
+diag_finish_kernel(int64_t count, const double *__restrict__ part, T *__restrict__ dshift,
                    int accumulate) {
     __shared__ double red[33];
     const int b = blockIdx.x;
     double s = 0.0;
-    for (int t = threadIdx.x; t < ntiles; t += kEdgeThreads) s += part[(int64_t)b * ntiles + t];
+    for (int64_t t = threadIdx.x; t < count; t += kEdgeThreads) s += part[(int64_t)b * count + t];
     s = block_sum<kEdgeThreads>(s, red);
     if (threadIdx.x == 0) dshift[b] = accumulate ? dshift[b] + (T)s : (T)s;
 }
@@ -206,7 +208,9 @@ unsigned grid_of(int64_t count) { return (unsigned)((count + kEdgeThreads - 1) /
 
 template <typename T, bool FROM_G>
 sla_status edge_grad(const Edges *p, const T *G, const T *lam, const T *x, T *dw, T *dshift,
-                     int accumulate, void *ws, size_t ws_bytes, cudaStream_t s) {
+                     int flags, void *ws, size_t ws_bytes, cudaStream_t s) {
+    const int accumulate = (flags & SLA_GRAD_ACCUMULATE) != 0;
+    const bool shared = (flags & SLA_GRAD_SHIFT_SHARED) != 0;
     const Csr *h = p->h;
     const int B = h->batch, n = h->n_rows;
     SLA_REQUIRE(B <= 65535, "sla_laplacian_grad: batch %d exceeds 65535", B);
@@ -227,7 +231,10 @@ sla_status edge_grad(const Edges *p, const T *G, const T *lam, const T *x, T *dw
                 n, h->nnz, p->ntiles, h->diagpos, G, lam, x, part);
             SLA_CHECK_LAUNCH();
         }
-        diag_finish_kernel<T><<<B, kEdgeThreads, 0, s>>>(p->ntiles, part, dshift, accumulate);
+        if (shared)
+            diag_finish_kernel<T><<<1, kEdgeThreads, 0, s>>>((int64_t)B * p->ntiles, part, dshift, accumulate);
+        else
+            diag_finish_kernel<T><<<B, kEdgeThreads, 0, s>>>(p->ntiles, part, dshift, accumulate);
         SLA_CHECK_LAUNCH();
     }
     return SLA_OK;
@@ -252,6 +259,7 @@ using namespace sla;
 extern "C" sla_status sla_edges_create(sla_csr_t hh, int64_t n_edges, const int32_t *ei,
                                        const int32_t *ej, int64_t *check, void *stream,
                                        sla_edges_t *out) {
+    SLA_RANGE("sla_edges_create");
     clear_error();
     if (check) *check = 0;
     SLA_REQUIRE(out != nullptr, "sla_edges_create: NULL out");
@@ -333,6 +341,7 @@ extern "C" sla_status sla_edges_destroy(sla_edges_t e) {
 
 extern "C" sla_status sla_laplacian_assemble(sla_edges_t ee, const void *w, const void *shift,
                                              void *vals, void *stream) {
+    SLA_RANGE("sla_laplacian_assemble");
     clear_error();
     const Edges *p = reinterpret_cast<const Edges *>(ee);
     SLA_REQUIRE(p != nullptr, "sla_laplacian_assemble: NULL plan");
@@ -360,31 +369,37 @@ extern "C" size_t sla_edges_workspace_bytes(sla_edges_t ee) {
 }
 
 extern "C" sla_status sla_laplacian_grad_values(sla_edges_t ee, const void *G, void *dw, void *dshift,
-                                                int32_t accumulate, void *ws, size_t ws_bytes,
+                                                int32_t flags, void *ws, size_t ws_bytes,
                                                 void *stream) {
+    SLA_RANGE("sla_laplacian_grad_values");
     clear_error();
+    SLA_REQUIRE((flags & ~(int32_t)(SLA_GRAD_ACCUMULATE | SLA_GRAD_SHIFT_SHARED)) == 0,
+                "sla_laplacian_grad_values: unknown flags 0x%x", (unsigned)flags);
     const Edges *p = reinterpret_cast<const Edges *>(ee);
     SLA_REQUIRE(p != nullptr, "sla_laplacian_grad_values: NULL plan");
     SLA_REQUIRE(G != nullptr || p->h->nnz == 0, "sla_laplacian_grad_values: NULL G");
     cudaStream_t s = as_stream(stream);
     if (p->h->dtype == SLA_F64)
         return edge_grad<double, true>(p, (const double *)G, nullptr, nullptr, (double *)dw,
-                                       (double *)dshift, accumulate, ws, ws_bytes, s);
+                                       (double *)dshift, flags, ws, ws_bytes, s);
     return edge_grad<float, true>(p, (const float *)G, nullptr, nullptr, (float *)dw, (float *)dshift,
-                                  accumulate, ws, ws_bytes, s);
+                                  flags, ws, ws_bytes, s);
 }
 
 extern "C" sla_status sla_laplacian_grad(sla_edges_t ee, const void *lambda, const void *x, void *dw,
-                                         void *dshift, int32_t accumulate, void *ws, size_t ws_bytes,
+                                         void *dshift, int32_t flags, void *ws, size_t ws_bytes,
                                          void *stream) {
+    SLA_RANGE("sla_laplacian_grad");
     clear_error();
+    SLA_REQUIRE((flags & ~(int32_t)(SLA_GRAD_ACCUMULATE | SLA_GRAD_SHIFT_SHARED)) == 0,
+                "sla_laplacian_grad: unknown flags 0x%x", (unsigned)flags);
     const Edges *p = reinterpret_cast<const Edges *>(ee);
     SLA_REQUIRE(p != nullptr, "sla_laplacian_grad: NULL plan");
     SLA_REQUIRE((lambda && x) || p->h->n_rows == 0, "sla_laplacian_grad: NULL lambda or x");
     cudaStream_t s = as_stream(stream);
     if (p->h->dtype == SLA_F64)
         return edge_grad<double, false>(p, nullptr, (const double *)lambda, (const double *)x,
-                                        (double *)dw, (double *)dshift, accumulate, ws, ws_bytes, s);
+                                        (double *)dw, (double *)dshift, flags, ws, ws_bytes, s);
     return edge_grad<float, false>(p, nullptr, (const float *)lambda, (const float *)x, (float *)dw,
-                                   (float *)dshift, accumulate, ws, ws_bytes, s);
+                                   (float *)dshift, flags, ws, ws_bytes, s);
 }

@@ -192,11 +192,54 @@ using namespace sla;
 
 extern "C" const char *sla_last_error_string(void) { return g_error.c_str(); }
 
-extern "C" const char *sla_version(void) { return "sla 0.1.0 (sm_100a)"; }
+extern "C" const char *sla_version(void) {
+    return SLA_DEBUG_BOUNDS ? "sla 0.2.0 (sm_100a, bounds-checking build)" : "sla 0.2.0 (sm_100a)";
+}
+
+#if SLA_DEBUG_BOUNDS
+namespace sla {
+// Readers of every translation unit's bounds record, registered at load time.
+static std::vector<DbgReader> &dbg_readers() {
+    static std::vector<DbgReader> r;
+    return r;
+}
+int dbg_register(DbgReader f) {
+    dbg_readers().push_back(f);
+    return (int)dbg_readers().size();
+}
+}  // namespace sla
+#endif
+
+extern "C" sla_status sla_debug_bounds_report(uint64_t *violations, int32_t *first_code,
+                                              int64_t *first_index, int32_t reset) {
+    clear_error();
+#if SLA_DEBUG_BOUNDS
+    unsigned long long count = 0, first = ~0ull;
+    for (DbgReader f : dbg_readers()) {
+        unsigned long long c = 0, fi = ~0ull;
+        SLA_CHECK_CUDA(f(&c, &fi, reset != 0));
+        count += c;
+        if (fi < first) first = fi;
+    }
+    if (violations) *violations = count;
+    if (first_code) *first_code = count ? (int32_t)(first >> 56) : 0;
+    if (first_index) *first_index = count ? (int64_t)(first & ((1ull << 56) - 1)) : -1;
+    return SLA_OK;
+#else
+    (void)reset;
+    if (violations) *violations = 0;
+    if (first_code) *first_code = 0;
+    if (first_index) *first_index = -1;
+    set_error("sla_debug_bounds_report: this library was built without SLA_DEBUG_BOUNDS "
+              "(load libsla_debug_bounds.so)");
+    return SLA_ERR_UNSUPPORTED;
+#endif
+}
 
 extern "C" sla_status sla_csr_check(int32_t n_rows, int32_t n_cols, int64_t nnz,
                                     const int32_t *rowptr, const int32_t *colind,
                                     int32_t need_diag, int64_t *result, void *stream) {
+    SLA_RANGE("sla_csr_check");
     clear_error();
     SLA_REQUIRE(n_rows >= 0 && n_cols >= 0 && nnz >= 0 && nnz <= INT_MAX,
                 "sla_csr_check: bad sizes n_rows=%d n_cols=%d nnz=%lld", n_rows, n_cols,
@@ -218,6 +261,7 @@ extern "C" sla_status sla_csr_create(int32_t n_rows, int32_t n_cols, int64_t nnz
                                      const int32_t *rowptr, const int32_t *colind,
                                      int32_t batch, sla_dtype dtype, uint32_t flags,
                                      void *stream, sla_csr_t *out) {
+    SLA_RANGE("sla_csr_create");
     clear_error();
     return create_handle(n_rows, n_cols, nnz, rowptr, colind, batch, dtype, flags, stream, out, false);
 }
@@ -226,6 +270,7 @@ extern "C" sla_status sla_csr_list_create(int32_t n_items, const int32_t *item_r
                                           int64_t nnz, const int32_t *rowptr, const int32_t *colind,
                                           sla_dtype dtype, uint32_t flags, void *stream,
                                           sla_csr_t *out) {
+    SLA_RANGE("sla_csr_list_create");
     clear_error();
     SLA_REQUIRE(out != nullptr, "sla_csr_list_create: NULL out");
     *out = nullptr;
@@ -391,7 +436,10 @@ sla_status create_handle(int32_t n_rows, int32_t n_cols, int64_t nnz, const int3
         if (st != SLA_OK) return fail(st);
         const char *sv = getenv("SLA_SELL");
         if (h->lanes == 1 && n_rows > 0 && !(sv && sv[0] == '0')) {
-            st = build_sell(h, s);
+            // rows sorted within windows only for solver variants that keep q by row and
+            // whose windows never straddle a tile (the interleaved batch solver does not)
+            const bool sort_ok = !h->onchip && h->il_blocks == 0 && h->tile_rows % kSellSortWindow == 0;
+            st = build_sell(h, sort_ok, s);
             if (st != SLA_OK) return fail(st);
         }
     }
@@ -415,6 +463,7 @@ extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     cudaFree(h->sell_ptr);
     cudaFree(h->sell_cols);
     cudaFree(h->sell_map);
+    cudaFree(h->sell_perm);
     cudaFree(h->dep_lo);
     cudaFree(h->dep_hi);
     cudaFree(h->seg);
@@ -439,9 +488,9 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_blocks = h->grid_blocks;
     p->block_fits = h->block_fits ? 1 : 0;
     p->has_transpose = h->has_transpose ? 1 : 0;
-    p->grid_onchip = h->onchip ? (h->grid2 && h->has_sell ? 2 : 1) : 0;
+    p->grid_onchip = h->onchip ? (h->grid2 && h->has_sell ? 2 : 1) : (h->rqs ? 3 : 0);
     p->grid_tile_rows = h->tile_rows;
-    p->sliced = h->has_sell ? 1 : 0;
+    p->sliced = h->has_sell ? (h->sell_w > 0 ? 2 : (h->sell_perm ? 3 : 1)) : 0;
     p->block_resident = h->block_mres ? 1 : 0;
     p->cluster_fits = h->cluster_fits ? 1 : 0;
     p->n_items = h->n_items;
@@ -454,6 +503,7 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
 extern "C" sla_status sla_csr_transpose_pattern(sla_csr_t hh, const int32_t **rowptrT,
                                                 const int32_t **colindT, const int32_t **perm,
                                                 void *stream) {
+    SLA_RANGE("sla_csr_transpose_pattern");
     clear_error();
     Csr *h = reinterpret_cast<Csr *>(hh);
     SLA_REQUIRE(h && rowptrT && colindT && perm, "sla_csr_transpose_pattern: NULL argument");

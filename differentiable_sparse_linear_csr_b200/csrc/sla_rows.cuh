@@ -24,15 +24,20 @@ __device__ __forceinline__ unsigned subwarp_mask() {
 
 // sum_{t in row i} vals[t] * v[colind[t]]; lane in [0, LANES).  With LANES > 1
 // the partial sums are combined by a fixed xor tree, so the result is
-// deterministic and identical on every lane of the sub-warp.
+// deterministic and identical on every lane of the sub-warp.  ncols (the length
+// of v) and nent (of vals and colind) bound the indices in the bounds-checking
+// build and are unused otherwise.
 template <typename T, int LANES>
 __device__ __forceinline__ T row_dot(const int32_t *__restrict__ rowptr,
                                      const int32_t *__restrict__ colind,
                                      const T *__restrict__ vals, const T *v, int i,
-                                     int lane) {
+                                     int lane, int ncols, int64_t nent) {
     const int t0 = __ldg(rowptr + i), t1 = __ldg(rowptr + i + 1);
     T s = T(0);
-    for (int t = t0 + lane; t < t1; t += LANES) s += __ldg(vals + t) * v[__ldg(colind + t)];
+    for (int t = t0 + lane; t < t1; t += LANES) {
+        const int tt = SLA_IDX(t, nent, kBndEntry);
+        s += __ldg(vals + tt) * v[SLA_IDX(__ldg(colind + tt), ncols, kBndColumn)];
+    }
     if constexpr (LANES > 1) {
         const unsigned m = subwarp_mask<LANES>();
 #pragma unroll
@@ -44,10 +49,14 @@ __device__ __forceinline__ T row_dot(const int32_t *__restrict__ rowptr,
 // Same product with every array in shared memory (plain loads).
 template <typename T, int LANES>
 __device__ __forceinline__ T row_dot_shared(const int32_t *rowptr, const int32_t *colind,
-                                            const T *vals, const T *v, int i, int lane) {
+                                            const T *vals, const T *v, int i, int lane,
+                                            int ncols, int64_t nent) {
     const int t0 = rowptr[i], t1 = rowptr[i + 1];
     T s = T(0);
-    for (int t = t0 + lane; t < t1; t += LANES) s += vals[t] * v[colind[t]];
+    for (int t = t0 + lane; t < t1; t += LANES) {
+        const int tt = SLA_IDX(t, nent, kBndLocal);
+        s += vals[tt] * v[SLA_IDX(colind[tt], ncols, kBndLocal)];
+    }
     if constexpr (LANES > 1) {
         const unsigned m = subwarp_mask<LANES>();
 #pragma unroll
@@ -63,11 +72,14 @@ __device__ __forceinline__ T row_dot_perm(const int32_t *__restrict__ rowptr,
                                           const int32_t *__restrict__ colind,
                                           const int32_t *__restrict__ perm,
                                           const T *__restrict__ vals, const T *v, int i,
-                                          int lane) {
+                                          int lane, int ncols, int64_t nent) {
     const int t0 = __ldg(rowptr + i), t1 = __ldg(rowptr + i + 1);
     T s = T(0);
-    for (int t = t0 + lane; t < t1; t += LANES)
-        s += __ldg(vals + __ldg(perm + t)) * v[__ldg(colind + t)];
+    for (int t = t0 + lane; t < t1; t += LANES) {
+        const int tt = SLA_IDX(t, nent, kBndEntry);
+        s += __ldg(vals + SLA_IDX(__ldg(perm + tt), nent, kBndEntry)) *
+             v[SLA_IDX(__ldg(colind + tt), ncols, kBndColumn)];
+    }
     if constexpr (LANES > 1) {
         const unsigned m = subwarp_mask<LANES>();
 #pragma unroll
@@ -76,52 +88,100 @@ __device__ __forceinline__ T row_dot_perm(const int32_t *__restrict__ rowptr,
     return s;
 }
 
-// Row i of the sliced layout (see sla_sell.cu) times v, one thread per row:
-// entries in stored order, then the slice's zero padding (which adds nothing).
-// R rows i0, i0 + stride, ... are interleaved so that their loads overlap;
-// rows >= row_end are skipped.
-// Loads of the sliced layout's entries.  With STREAM the load bypasses L1
-// (ld.global.nc.L1::no_allocate): in the solver whose vectors live in HBM the
-// matrix streams through once per iteration and L1 is better left to the
-// gathered vector; where the matrix stays in L2 the default allocating load is
-// faster (a slice step uses half a 128-byte line, the next step the other half).
-template <bool STREAM, typename T>
+// Loads of the sliced layout's entries, by MODE:
+//   0  the default allocating read-only load (the matrix stays in L2 and L1);
+//   1  ld.global.nc.L1::no_allocate: in the solver whose vectors live in HBM the
+//      matrix streams through once per iteration and L1 is better left to the
+//      gathered vector; where the matrix stays in L2 the allocating load is
+//      faster (a slice step uses half a 128-byte line, the next step the other);
+//   2  as 1, with an L2 evict-first policy, so that the streamed matrix leaves
+//      L2 before the vectors;
+//   3  as 1, asking L2 to fetch the whole 256-byte block on a miss.
+__device__ __forceinline__ unsigned long long l2_evict_first_policy() {
+    unsigned long long pol;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+template <int MODE, typename T>
 __device__ __forceinline__ T sell_load(const T *p) {
-    if constexpr (STREAM) {
-        if constexpr (sizeof(T) == 8) {
-            double v;
-            asm volatile("ld.global.nc.L1::no_allocate.f64 %0, [%1];" : "=d"(v) : "l"(p));
-            return (T)v;
-        } else if constexpr (std::is_same<T, float>::value) {
-            float v;
-            asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
-            return v;
-        } else {
-            int v;
-            asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
-            return (T)v;
-        }
-    } else {
+    static_assert(sizeof(T) == 4 || sizeof(T) == 8, "4- or 8-byte entries");
+    if constexpr (MODE == 0) {
         return __ldg(p);
+    } else if constexpr (sizeof(T) == 8) {
+        double v;
+        if constexpr (MODE == 1)
+            asm volatile("ld.global.nc.L1::no_allocate.f64 %0, [%1];" : "=d"(v) : "l"(p));
+        else if constexpr (MODE == 2)
+            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f64 %0, [%1], %2;"
+                         : "=d"(v) : "l"(p), "l"(l2_evict_first_policy()));
+        else
+            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.f64 %0, [%1];" : "=d"(v) : "l"(p));
+        return (T)v;
+    } else if constexpr (std::is_same<T, float>::value) {
+        float v;
+        if constexpr (MODE == 1)
+            asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+        else if constexpr (MODE == 2)
+            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;"
+                         : "=f"(v) : "l"(p), "l"(l2_evict_first_policy()));
+        else
+            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.f32 %0, [%1];" : "=f"(v) : "l"(p));
+        return v;
+    } else {
+        int v;
+        if constexpr (MODE == 1)
+            asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
+        else if constexpr (MODE == 2)
+            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.s32 %0, [%1], %2;"
+                         : "=r"(v) : "l"(p), "l"(l2_evict_first_policy()));
+        else
+            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.s32 %0, [%1];" : "=r"(v) : "l"(p));
+        return (T)v;
     }
+}
+
+// Asks L2 to fetch [p, p + bytes) from memory ahead of use (a bulk prefetch
+// issued by one thread; no registers or shared memory wait for it).  p must be
+// 16-byte aligned and bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, unsigned bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// First slot and width of row i's slice: computed when every slice has the
+// same width uw (no load), else read from the slice offsets.
+__device__ __forceinline__ void sell_slice(const int32_t *__restrict__ sptr, int i, int uw, int &base,
+                                           int &w) {
+    const int sl = i / kSellRows;
+    int b0;
+    if (uw > 0) {
+        b0 = sl * kSellRows * uw;
+        w = uw;
+    } else {
+        b0 = __ldg(sptr + sl);
+        w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
+    }
+    base = b0 + i % kSellRows;
 }
 
 // Row i of the sliced layout (see sla_sell.cu) times v, one thread per row:
 // the row's entries in stored order, then the slice's zero padding (which adds
 // nothing), so the sum equals row_dot<T, 1>.  One row at a time per thread:
-// interleaving a thread's rows spreads its gathers of v and measured slower.
-template <bool STREAM, typename T>
+// interleaving a thread's rows spreads its gathers of v and measured slower,
+// and so did loading a row's entries into registers before gathering (the
+// registers spill at the solver's 64-register budget).  uw > 0: every slice is
+// uw wide (no slice offsets read).
+template <int STREAM, typename T>
 __device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
                                       const int32_t *__restrict__ cols,
-                                      const T *__restrict__ vals, const T *v, int i) {
-    const int sl = i / kSellRows;
-    const int b0 = __ldg(sptr + sl);
-    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
-    const int base = b0 + i % kSellRows;
+                                      const T *__restrict__ vals, const T *v, int i,
+                                      int ncols, int64_t nslots, int uw) {
+    int base, w;
+    sell_slice(sptr, i, uw, base, w);
     T s = T(0);
     for (int k = 0; k < w; ++k) {
-        const int t = base + k * kSellRows;
-        s += sell_load<STREAM>(vals + t) * v[sell_load<STREAM>(cols + t)];
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        s += sell_load<STREAM>(vals + t) * v[SLA_IDX(sell_load<STREAM>(cols + t), ncols, kBndColumn)];
     }
     return s;
 }
@@ -132,7 +192,7 @@ template <typename T> struct SellRec;
 template <> struct __align__(16) SellRec<double> { double v; int32_t c, pad; };
 template <> struct __align__(8) SellRec<float> { float v; int32_t c; };
 
-template <bool STREAM, typename T>
+template <int STREAM, typename T>
 __device__ __forceinline__ void sell_rec_load(const SellRec<T> *p, T &v, int &c) {
     if constexpr (sizeof(T) == 8) {
         int4 u;
@@ -155,9 +215,9 @@ __device__ __forceinline__ void sell_rec_load(const SellRec<T> *p, T &v, int &c)
 }
 
 // sell_row over packed records: same entries, order and rounding.
-template <bool STREAM, typename T>
+template <int STREAM, typename T>
 __device__ __forceinline__ T sell_row_rec(const int32_t *__restrict__ sptr, const SellRec<T> *__restrict__ rec,
-                                          const T *v, int i) {
+                                          const T *v, int i, int ncols, int64_t nslots) {
     const int sl = i / kSellRows;
     const int b0 = __ldg(sptr + sl);
     const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
@@ -166,8 +226,8 @@ __device__ __forceinline__ T sell_row_rec(const int32_t *__restrict__ sptr, cons
     for (int k = 0; k < w; ++k) {
         T a;
         int c;
-        sell_rec_load<STREAM>(rec + base + k * kSellRows, a, c);
-        s += a * v[c];
+        sell_rec_load<STREAM>(rec + SLA_IDX(base + k * kSellRows, nslots, kBndEntry), a, c);
+        s += a * v[SLA_IDX(c, ncols, kBndColumn)];
     }
     return s;
 }
@@ -179,15 +239,13 @@ template <typename T>
 __device__ __forceinline__ T sell_row_dir(const int32_t *__restrict__ sptr,
                                           const int32_t *__restrict__ cols,
                                           const T *__restrict__ vals, const T *z, const T *pprev,
-                                          T beta, int i) {
-    const int sl = i / kSellRows;
-    const int b0 = __ldg(sptr + sl);
-    const int w = (__ldg(sptr + sl + 1) - b0) / kSellRows;
-    const int base = b0 + i % kSellRows;
+                                          T beta, int i, int ncols, int64_t nslots, int uw) {
+    int base, w;
+    sell_slice(sptr, i, uw, base, w);
     T s = T(0);
     for (int k = 0; k < w; ++k) {
-        const int t = base + k * kSellRows;
-        const int c = __ldg(cols + t);
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        const int c = SLA_IDX(__ldg(cols + t), ncols, kBndColumn);
         T pj;
         if constexpr (sizeof(T) == 8) pj = __fma_rn(beta, pprev[c], z[c]);
         else pj = __fmaf_rn(beta, pprev[c], z[c]);

@@ -8,11 +8,44 @@
 // several rows in flight.  Padding entries point at the row itself with value
 // 0, which leaves the row sum unchanged: rows are still summed in stored order.
 // The values are laid out per solve (one gather pass) into the workspace.
+//
+// Two refinements, chosen at creation:
+//  - uniform width: when padding every slice to the widest row costs at most
+//    3 % of the entries (stencil and grid patterns), all slices get that width
+//    and the kernels compute a slice's first slot instead of reading it;
+//  - sorted windows (the SELL-C-sigma idea of Kreutzer, Hager, Wellein, Fehske
+//    and Bishop, 2014, with sigma = 32): for irregular row lengths, the rows of
+//    each aligned 32-row window are ordered by decreasing length (ties by row)
+//    before they are cut into slices, so rows of similar length share a slice
+//    and the padding shrinks (a 10-entry-mean kNN graph: 19 % -> 6 %).  A
+//    window is one warp's rows in the solver, so each warp still handles the
+//    same rows; sell_perm maps a position to its row.  Each row's entries keep
+//    their stored order, so its sum is unchanged.
+#include <cstdlib>
+
 #include "sla_common.cuh"
 
 namespace sla {
 
-__global__ void sell_width_kernel(int n, const int32_t *__restrict__ rowptr, unsigned *__restrict__ cnt) {
+// perm[pos] for the rows of each aligned 32-row window, longest first (ties by
+// row): one warp per window, each lane ranks its row against the other 31.
+__global__ void sell_sort_kernel(int n, const int32_t *__restrict__ rowptr, int32_t *__restrict__ perm) {
+    const int64_t win = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / kSellSortWindow;
+    const int lane = threadIdx.x % kSellSortWindow;
+    const int64_t i = win * kSellSortWindow + lane;
+    const int len = i < n ? rowptr[i + 1] - rowptr[i] : -1;
+    int rank = 0;
+    for (int j = 0; j < kSellSortWindow; ++j) {
+        const int lj = __shfl_sync(0xffffffffu, len, j);
+        rank += (lj > len) || (lj == len && j < lane);
+    }
+    if (i < n) perm[win * kSellSortWindow + rank] = (int32_t)i;
+}
+
+// Slots of each slice: 8 times the longest of its rows (the rows at its
+// positions when perm is given).
+__global__ void sell_width_kernel(int n, const int32_t *__restrict__ rowptr, const int32_t *__restrict__ perm,
+                                  unsigned *__restrict__ cnt) {
     const int64_t sl = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t nsl = ((int64_t)n + kSellRows - 1) / kSellRows;
     if (sl > nsl) return;
@@ -20,22 +53,27 @@ __global__ void sell_width_kernel(int n, const int32_t *__restrict__ rowptr, uns
     int w = 0;
     for (int l = 0; l < kSellRows; ++l) {
         const int64_t i = sl * kSellRows + l;
-        if (i < n) w = max(w, rowptr[i + 1] - rowptr[i]);
+        if (i < n) {
+            const int r = perm ? perm[i] : (int)i;
+            w = max(w, rowptr[r + 1] - rowptr[r]);
+        }
     }
     cnt[sl] = (unsigned)(w * kSellRows);
 }
 
 __global__ void sell_fill_kernel(int n, const int32_t *__restrict__ rowptr,
                                  const int32_t *__restrict__ colind, const int32_t *__restrict__ sptr,
-                                 int32_t *__restrict__ cols, int32_t *__restrict__ map) {
+                                 const int32_t *__restrict__ perm, int32_t *__restrict__ cols,
+                                 int32_t *__restrict__ map) {
     const int64_t sl = blockIdx.x * (int64_t)(blockDim.x / kSellRows) + threadIdx.x / kSellRows;
     const int l = threadIdx.x % kSellRows;
     const int64_t nsl = ((int64_t)n + kSellRows - 1) / kSellRows;
     if (sl >= nsl) return;
     const int64_t i = sl * kSellRows + l;
     const int base = sptr[sl], w = (sptr[sl + 1] - base) / kSellRows;
-    const int t0 = i < n ? rowptr[i] : 0, len = i < n ? rowptr[i + 1] - t0 : 0;
-    const int own = i < n ? (int)i : 0;
+    const int row = i < n ? (perm ? perm[i] : (int)i) : 0;
+    const int t0 = i < n ? rowptr[row] : 0, len = i < n ? rowptr[row + 1] - t0 : 0;
+    const int own = row;
     for (int k = 0; k < w; ++k) {
         const int slot = base + k * kSellRows + l;
         if (k < len) {
@@ -58,15 +96,51 @@ __global__ void sell_values_kernel(int64_t sell_nnz, int64_t nnz, int B, const i
         out[(int64_t)b * sell_nnz + slot] = t >= 0 ? vals[(int64_t)b * nnz + t] : T(0);
 }
 
-sla_status build_sell(Csr *h, cudaStream_t s) {
+// Every slice padded to the widest row: slice s starts at slot s * 8 * w.
+__global__ void sell_uniform_ptr_kernel(int64_t nsl, int w, int32_t *__restrict__ sptr) {
+    const int64_t sl = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (sl <= nsl) sptr[sl] = (int32_t)(sl * kSellRows * w);
+}
+
+sla_status build_sell(Csr *h, bool sort_ok, cudaStream_t s) {
     const int n = h->n_rows;
     const int64_t nsl = ((int64_t)n + kSellRows - 1) / kSellRows;
+    SLA_CHECK_CUDA(cudaMalloc(&h->sell_ptr, (size_t)(nsl + 1) * sizeof(int32_t)));
+    // Uniform width when padding every slice to the widest row costs at most 3 %
+    // of the entries (stencil and grid patterns): the kernels then compute a
+    // slice's first slot instead of reading it.  SLA_SELL_UNIFORM=0 turns it off.
+    const int64_t uslots = nsl * kSellRows * (int64_t)h->row_max;
+    const char *ue = getenv("SLA_SELL_UNIFORM");
+    if (h->row_max > 0 && uslots <= 0x7fffffffLL && (double)(uslots - h->nnz) <= 0.03 * (double)h->nnz &&
+        !(ue && ue[0] == '0')) {
+        sell_uniform_ptr_kernel<<<(unsigned)((nsl + 1 + 255) / 256), 256, 0, s>>>(nsl, h->row_max, h->sell_ptr);
+        SLA_CHECK_LAUNCH();
+        h->sell_w = h->row_max;
+        h->sell_nnz = uslots;
+        SLA_CHECK_CUDA(cudaMalloc(&h->sell_cols, (size_t)uslots * sizeof(int32_t)));
+        SLA_CHECK_CUDA(cudaMalloc(&h->sell_map, (size_t)uslots * sizeof(int32_t)));
+        constexpr int kThreads = 256;
+        const unsigned grid = (unsigned)((nsl + kThreads / kSellRows - 1) / (kThreads / kSellRows));
+        sell_fill_kernel<<<grid, kThreads, 0, s>>>(n, h->rowptr, h->colind, h->sell_ptr, nullptr,
+                                                   h->sell_cols, h->sell_map);
+        SLA_CHECK_LAUNCH();
+        h->has_sell = true;
+        return SLA_OK;
+    }
+    // Irregular rows: sort each 32-row window by length when the solver keeps q
+    // by row index (SLA_SELL_SORT=0 turns it off).
+    const char *se = getenv("SLA_SELL_SORT");
+    if (sort_ok && h->row_min != h->row_max && !(se && se[0] == '0')) {
+        SLA_CHECK_CUDA(cudaMalloc(&h->sell_perm, (size_t)n * sizeof(int32_t)));
+        const int64_t threads = ((int64_t)n + kSellSortWindow - 1) / kSellSortWindow * kSellSortWindow;
+        sell_sort_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(n, h->rowptr, h->sell_perm);
+        SLA_CHECK_LAUNCH();
+    }
     unsigned *cnt = nullptr;
     void *ws = nullptr;
-    SLA_CHECK_CUDA(cudaMalloc(&h->sell_ptr, (size_t)(nsl + 1) * sizeof(int32_t)));
     SLA_CHECK_CUDA(cudaMalloc(&cnt, (size_t)(nsl + 1) * sizeof(unsigned)));
     SLA_CHECK_CUDA(cudaMalloc(&ws, scan_ws_bytes(nsl + 1)));
-    sell_width_kernel<<<(unsigned)((nsl + 1 + 255) / 256), 256, 0, s>>>(n, h->rowptr, cnt);
+    sell_width_kernel<<<(unsigned)((nsl + 1 + 255) / 256), 256, 0, s>>>(n, h->rowptr, h->sell_perm, cnt);
     SLA_CHECK_LAUNCH();
     sla_status st = exclusive_scan(cnt, reinterpret_cast<unsigned *>(h->sell_ptr), nsl + 1, ws, s);
     unsigned total = 0;
@@ -82,7 +156,8 @@ sla_status build_sell(Csr *h, cudaStream_t s) {
     }
     if (total > 0x7fffffffu) {   // padded layout would overflow int32 offsets: keep CSR only
         cudaFree(h->sell_ptr);
-        h->sell_ptr = nullptr;
+        cudaFree(h->sell_perm);
+        h->sell_ptr = h->sell_perm = nullptr;
         return SLA_OK;
     }
     h->sell_nnz = total;
@@ -91,8 +166,8 @@ sla_status build_sell(Csr *h, cudaStream_t s) {
     SLA_CHECK_CUDA(cudaMalloc(&h->sell_map, z * sizeof(int32_t)));
     constexpr int kThreads = 256;
     const unsigned grid = (unsigned)((nsl + kThreads / kSellRows - 1) / (kThreads / kSellRows));
-    sell_fill_kernel<<<grid, kThreads, 0, s>>>(n, h->rowptr, h->colind, h->sell_ptr, h->sell_cols,
-                                               h->sell_map);
+    sell_fill_kernel<<<grid, kThreads, 0, s>>>(n, h->rowptr, h->colind, h->sell_ptr, h->sell_perm,
+                                               h->sell_cols, h->sell_map);
     SLA_CHECK_LAUNCH();
     h->has_sell = true;
     return SLA_OK;

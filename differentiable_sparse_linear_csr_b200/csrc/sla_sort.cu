@@ -360,6 +360,7 @@ extern "C" sla_status sla_csr_transpose(int32_t n_rows, int32_t n_cols, int64_t 
                                         int32_t batch, sla_dtype dtype, const void *vals,
                                         int32_t *rowptrT, int32_t *colindT, void *valsT,
                                         int32_t *perm, void *ws, size_t ws_bytes, void *stream) {
+    SLA_RANGE("sla_csr_transpose");
     clear_error();
     SLA_REQUIRE(n_rows >= 0 && n_cols >= 0 && nnz >= 0 && nnz <= 0x7fffffff,
                 "sla_csr_transpose: bad sizes");
@@ -394,6 +395,7 @@ extern "C" sla_status sla_csr_from_coo(int32_t n_rows, int32_t n_cols, int64_t n
                                        sla_dtype dtype, const void *val, int32_t *rowptr,
                                        int32_t *colind, void *val_out, int32_t *slot,
                                        int64_t *nnz_out, void *ws, size_t ws_bytes, void *stream) {
+    SLA_RANGE("sla_csr_from_coo");
     clear_error();
     SLA_REQUIRE(n_rows >= 0 && n_cols >= 0 && nnz_in >= 0 && nnz_in < 0x7fffffff,
                 "sla_csr_from_coo: bad sizes");

@@ -129,13 +129,19 @@ typedef struct {
     int32_t grid_onchip;      /* 1 if the grid solver keeps x, r, M^-1 on chip (else in HBM);
                                  2 if, besides, a single system on the sliced layout runs
                                  the two-barrier form (directions formed while gathered);
-                                 the environment variables SLA_GRID_ONCHIP=0 and
-                                 SLA_GRID2=0, read at creation, turn these variants off */
+                                 3 if it keeps r and q on chip and x, M^-1 in HBM (tiles
+                                 too large for three vectors on chip);
+                                 the environment variables SLA_GRID_ONCHIP=0, SLA_GRID2=0
+                                 and SLA_GRID_RQS=0, read at creation, turn these variants
+                                 off (SLA_GRID_ONCHIP=2 leaves only variant 3) */
     int32_t grid_tile_rows;   /* rows of one grid-solver tile (SLA_SELL_PACK=1, read at each
                                  solve, makes the sliced SpMV read value-and-column records,
                                  one load an entry; off by default, see the design notes) */
     int32_t sliced;           /* 1 if the grid solver uses the 8-row sliced layout (one
-                                 extra value-gather kernel per solve) */
+                                 extra value-gather kernel per solve); 2 if, besides,
+                                 every slice is padded to the widest row (padding at most
+                                 3 % of the entries; SLA_SELL_UNIFORM=0, read at creation,
+                                 turns this off) */
     int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
                                  system in shared memory as well as its vectors */
     int32_t cluster_fits;     /* 1 if one system fits the cluster solver */
@@ -234,6 +240,18 @@ sla_status sla_grad_values(sla_csr_t h, const void *lambda, const void *x, void 
                            int32_t accumulate, void *stream);
 
 /*
+ * Value gradient of the matrix-vector product ("Methodology" 1, `.matvec`, as an
+ * autograd operation): for y_b = A_b x_b and an incoming gradient gy_b = dL/dy_b,
+ * dL/dA_ij = gy_i * x_j on the stored entries only:  grad_b[t] = gy_b[i] *
+ * x_b[colind[t]] for entry t of row i, or grad_b[t] += that value when
+ * accumulate != 0.  gy [B][n_rows], x [B][n_cols], grad [B][nnz]; device.
+ * Each entry is one rounded product (sla_grad_values with lambda = gy gives
+ * its exact negation).
+ */
+sla_status sla_matvec_grad_values(sla_csr_t h, const void *gy, const void *x, void *grad,
+                                  int32_t accumulate, void *stream);
+
+/*
  * Transpose of a batched CSR matrix by a stable sort on the column index:
  * row c of A^T lists the entries of column c in increasing row order; values
  * are moved, never combined; perm[s] is the A-position of A^T's entry s.
@@ -291,9 +309,10 @@ sla_status sla_csr_check(int32_t n_rows, int32_t n_cols, int64_t nnz,
  * words, partial sums, diagonal positions, the r, p, q, M^-1 vectors) lives in
  * one static device array of 16 MiB that every GPU loading this library keeps
  * until the process exits.
- *   - The first call on a device performs a one-time set-up (it looks up the
- *     array's device address with that device current); make that first call
- *     before any stream capture.
+ *   - Every call looks up the array's device address in the caller's current
+ *     context (so a context switch or a device reset between calls is safe);
+ *     the first call in a context also loads the library's device code into
+ *     it, so make that first call before any stream capture.
  *   - Sizes whose scratch exceeds 16 MiB (about 4 + 4*sizeof(T) bytes per row
  *     and system, plus 32 bytes per tile) are rejected with SLA_ERR_INVALID
  *     and a message giving both sizes; it never allocates, not even then.
@@ -378,20 +397,45 @@ sla_status sla_laplacian_assemble(sla_edges_t e, const void *w, const void *shif
 /* Workspace (256-byte aligned) of the two gradient calls below. */
 size_t sla_edges_workspace_bytes(sla_edges_t e);
 
-/* dw (device [B][E]) and dshift (device [B], may be NULL) from G (device
- * [B][nnz]) by the chain rule above; with accumulate != 0 they are added to
- * dw / dshift.  dw is bit-exact (four entries added in the stated order);
- * dshift is accumulated in double over a fixed tree and rounded once. */
+/* Flags of the two gradient calls below. */
+enum {
+    SLA_GRAD_ACCUMULATE = 1u,    /* add to dw / dshift instead of overwriting them */
+    SLA_GRAD_SHIFT_SHARED = 2u   /* one shift serves every system: dshift is device [1]
+                                    and receives dL/ds summed over all systems */
+};
+
+/* dw (device [B][E]) and dshift (device [B], or [1] with SLA_GRAD_SHIFT_SHARED;
+ * may be NULL) from G (device [B][nnz]) by the chain rule above.  dw is
+ * bit-exact (four entries added in the stated order); dshift is accumulated in
+ * double over a fixed tree (over every system's diagonal with
+ * SLA_GRAD_SHIFT_SHARED) and rounded once.  flags: SLA_GRAD_*. */
 sla_status sla_laplacian_grad_values(sla_edges_t e, const void *G, void *dw, void *dshift,
-                                     int32_t accumulate, void *ws, size_t ws_bytes, void *stream);
+                                     int32_t flags, void *ws, size_t ws_bytes, void *stream);
 
 /* The same with G = -lambda x^T on the pattern (what sla_grad_values would
  * write), without forming G: each G entry is rounded exactly as
  * sla_grad_values rounds it, so dw equals sla_grad_values followed by
  * sla_laplacian_grad_values bit for bit.  lambda, x: device [B][n]. */
 sla_status sla_laplacian_grad(sla_edges_t e, const void *lambda, const void *x, void *dw,
-                              void *dshift, int32_t accumulate, void *ws, size_t ws_bytes,
+                              void *dshift, int32_t flags, void *ws, size_t ws_bytes,
                               void *stream);
+
+/*
+ * Bounds record of the bounds-checking build (libsla_debug_bounds.so, compiled
+ * with SLA_DEBUG_BOUNDS=1).  There is no counterpart on the pages: this build
+ * stands in for a memory checker.  Its kernels check every index they take from
+ * the pattern (gathered columns, entry positions, diagonal positions, edge
+ * slots) and every shared-memory or cluster-rank index derived from one before
+ * using it; a bad index is recorded and replaced by 0, so the access stays in
+ * bounds and no kernel traps.  This call waits for the device, then returns
+ * the number of violations since the last reset (*violations), the smallest
+ * code (1 column, 2 entry, 3 diagonal, 4 shared-memory or cluster index,
+ * 5 edge; 0 if none) and that code's smallest index (-1 if none); with
+ * reset != 0 it clears the record.  Any output pointer (host) may be NULL.
+ * The regular library returns SLA_ERR_UNSUPPORTED.
+ */
+sla_status sla_debug_bounds_report(uint64_t *violations, int32_t *first_code, int64_t *first_index,
+                                   int32_t reset);
 
 /* Message for the last non-OK status on this host thread ("" if none). */
 const char *sla_last_error_string(void);

@@ -53,6 +53,8 @@ def test_host_side_argument_errors_need_no_gpu():
     assert st == L.SLA_ERR_INVALID and "square" in L.sla_last_error_string()
     assert lib.sla_spmv(None, None, None, None, 0, 1.0, 0.0, None) == L.SLA_ERR_INVALID
     assert lib.sla_grad_values(None, None, None, None, 0, None) == L.SLA_ERR_INVALID
+    assert lib.sla_matvec_grad_values(None, None, None, None, 0, None) == L.SLA_ERR_INVALID
+    assert "sla_matvec_grad_values" in L.sla_last_error_string()
     opts = L.make_opts()
     info = L.make_info()
     assert lib.sla_cg_solve(None, None, None, None, ctypes.byref(opts), info, None, 0, None) == L.SLA_ERR_INVALID
@@ -67,6 +69,13 @@ def test_host_side_argument_errors_need_no_gpu():
     assert lib.sla_laplacian_assemble(None, None, None, None, None) == L.SLA_ERR_INVALID
     assert lib.sla_laplacian_grad_values(None, None, None, None, 0, None, 0, None) == L.SLA_ERR_INVALID
     assert lib.sla_laplacian_grad(None, None, None, None, None, 0, None, 0, None) == L.SLA_ERR_INVALID
+    for fn in (lib.sla_laplacian_grad_values, lib.sla_laplacian_grad):
+        args = [None] * (8 if fn is lib.sla_laplacian_grad_values else 9)
+        fl = 4 if fn is lib.sla_laplacian_grad_values else 5
+        args[fl], args[fl + 2] = 4, 0           # a flag bit beyond ACCUMULATE | SHIFT_SHARED
+        assert fn(*args) == L.SLA_ERR_INVALID and "flags" in L.sla_last_error_string()
+        args[fl] = L.SLA_GRAD_ACCUMULATE | L.SLA_GRAD_SHIFT_SHARED
+        assert fn(*args) == L.SLA_ERR_INVALID and "plan" in L.sla_last_error_string()
     assert lib.sla_edges_workspace_bytes(None) == 0
     assert lib.sla_edges_destroy(None) == L.SLA_OK
 
@@ -135,3 +144,20 @@ def test_list_create_argument_errors_need_no_gpu():
     assert "item_rows" in L.sla_last_error_string()
     assert lib.sla_csr_list_create(2, ctypes.c_void_p(256), 4, 0, ctypes.c_void_p(256), None, 0, 0, None,
                                    None) == L.SLA_ERR_INVALID
+
+
+def test_bounds_report_needs_the_bounds_checking_build():
+    """The regular library declines the report; the bounds-checking build loads
+    without a GPU, exports the same symbols and says what it is."""
+    v, c, i = ctypes.c_uint64(7), ctypes.c_int32(7), ctypes.c_int64(7)
+    st = L.lib().sla_debug_bounds_report(ctypes.byref(v), ctypes.byref(c), ctypes.byref(i), 0)
+    assert st == L.SLA_ERR_UNSUPPORTED and "SLA_DEBUG_BOUNDS" in L.sla_last_error_string()
+    assert (v.value, c.value, i.value) == (0, 0, -1)
+    path = os.path.join(ROOT, "differentiable_sparse_linear_csr_b200", "libsla_debug_bounds.so")
+    if not os.path.exists(path):
+        pytest.skip("bounds-checking library not built")
+    dbg = ctypes.CDLL(path)
+    missing = [n for n in _declared_functions() if not hasattr(dbg, n)]
+    assert not missing, missing
+    dbg.sla_version.restype = ctypes.c_char_p
+    assert b"bounds-checking" in dbg.sla_version()

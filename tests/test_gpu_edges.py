@@ -216,6 +216,33 @@ def test_edge_solve_forward_and_backward_match_the_oracle(dtype):
     assert same_bits(H(st2.grad), H(st.grad))
 
 
+def test_shared_shift_gradient_is_the_sum_over_systems():
+    """One shift tensor of one element serving a batch of 3: the library sums
+    dL/dshift over the systems (SLA_GRAD_SHIFT_SHARED), through both the fused
+    edge solve and the assembly's own backward; the result equals the sum of the
+    oracle's per-system shift gradients, and both paths agree bit for bit."""
+    ei, ej = W.grid_edges((16, 16))
+    n, B = 256, 3
+    w = W.uniform(62, W.STREAM_WEIGHTS, B * ei.shape[0], 0.5, 2.0).reshape(B, -1)
+    b = W.normal(62, W.STREAM_B, B * n).reshape(B, n)
+    xs = W.uniform(62, W.STREAM_XSTAR, B * n, -1, 1).reshape(B, n)
+    rp, ci, _ = W.weighted_laplacian(n, ei, ej, w[0], 0.0)
+    A, E = _plan(rp, ci, ei, ej, B, torch.float64)
+    st = torch.tensor([2e-2], dtype=torch.float64, device=DEV, requires_grad=True)
+    x = E.solve(T(w), T(b), st, rtol=1e-12)
+    (0.5 * ((x - T(xs)) ** 2).sum()).backward()
+    vo = np.stack([O.laplacian_assemble(rp, ci, ei, ej, w[s], 2e-2) for s in range(B)])
+    xo, _ = O.pcg(rp, ci, vo, b, rtol=1e-12)
+    lo, _ = O.cg_adjoint(rp, ci, vo, xo - xs, rtol=1e-12)
+    _, dso = O.laplacian_grad_values(rp, ci, ei, ej, O.grad_values(rp, ci, lo, xo))
+    assert st.grad.shape == (1,)
+    assert abs(float(st.grad[0]) - dso.sum()) <= 1e-6 * np.abs(dso).sum()
+    st2 = torch.tensor([2e-2], dtype=torch.float64, device=DEV, requires_grad=True)
+    x2 = A.solve(E.assemble(T(w), st2), T(b), rtol=1e-12)
+    (0.5 * ((x2 - T(xs)) ** 2).sum()).backward()
+    assert same_bits(H(st2.grad), H(st.grad))
+
+
 def test_inverse_coefficient_learning_with_adam():
     """Edge conductivities of a 12x12 grid recovered from 8 observed solutions
     with a plain Adam loop through EdgeLaplacian.solve (the pages' end-to-end

@@ -1,12 +1,16 @@
 """Full-size workloads: the GPU path against the CPU oracle at the sizes and in
 the launch configuration the benchmark times.
 
-Element-by-element parity where the oracle finishes in reasonable time (the
-1024x1024 Poisson system at its fixed 1000 + 1000 iterations, fp64 and fp32;
-fixed iteration counts for the 3-D diffusion, the batch and the kNN graph);
-otherwise properties that hold at any size, computed with scipy from the GPU's
-outputs (true residual, adjoint and Euler identities, the gradient formula on
-sampled entries).  The oracle never receives a GPU result as input.
+Element by element against the oracle, solution, adjoint and value gradient:
+the 1024x1024 Poisson system at its fixed 1000 + 1000 iterations (fp64 and
+fp32); the 3-D diffusion at fixed counts and in the benchmark's tolerance mode
+at the GPU's own iteration counts (fp64 and fp32); every system of the batch;
+the kNN graph in both orders at a fixed count.  Besides, properties that hold
+at any size, computed with scipy from the GPU's outputs (true residual, adjoint
+and Euler identities, the gradient formula on sampled entries), for the
+tolerance-mode runs.  The oracle never receives a GPU result as input: where it
+runs the GPU's iteration count, it starts from the same inputs and iterates on
+its own.
 """
 import numpy as np
 import pytest
@@ -112,13 +116,51 @@ def test_c3_diffusion3d_fixed_and_tolerance():
     _properties(w, H(x)[0], H(lam)[0], H(G)[0], 1e-8, b[0], xs[0], v[0])
 
 
-def test_c3_diffusion3d_fp32_fixed():
+def test_c3_diffusion3d_tolerance_mode_elementwise_at_the_gpu_counts():
+    """The benchmark's run (PCG to 1e-8, adjoint to 1e-8, gradient), element by
+    element: the oracle runs exactly the GPU's forward and adjoint iteration
+    counts (the reading for ties at the tolerance) on its own iterates."""
+    w = W.c3_diffusion3d()
+    A = sla.CSR(T(w.rowptr), T(w.colind), symmetric=True)
+    v, b, xs = w.values, w.b, w.xstar
+    x, lam, G, fi, ai = _pipeline(A, T(v), T(b), T(xs), rtol=1e-8)
+    kf, ka = int(H(fi.iters)[0]), int(H(ai.iters)[0])
+    assert H(fi.status)[0] == L.SLA_CONVERGED and H(ai.status)[0] == L.SLA_CONVERGED
+    xo, _ = O.pcg(w.rowptr, w.colind, v[0], b[0], fixed_iters=kf)
+    lo, _ = O.cg_adjoint(w.rowptr, w.colind, v[0], xo - xs[0], fixed_iters=ka)
+    Go = O.grad_values(w.rowptr, w.colind, lo, xo)
+    assert rel(H(x)[0], xo) < TOL_X64
+    assert rel(H(lam)[0], lo) < TOL_G64
+    assert rel(H(G)[0], Go) < TOL_G64
+
+
+def test_c3_diffusion3d_fp32_forward_adjoint_gradient():
+    """fp32 at a fixed 200 + 200 iterations against the fp32 oracle: solution,
+    adjoint and value gradient element by element at the fp32 bar."""
     w = W.c3_diffusion3d()
     A = sla.CSR(T(w.rowptr), T(w.colind), dtype=torch.float32, symmetric=True)
-    v, b = w.values.astype(np.float32), w.b.astype(np.float32)
-    xo, _ = O.pcg(w.rowptr, w.colind, v[0], b[0], fixed_iters=200)
-    x, fi = A.cg(T(v), T(b), fixed_iters=200)
+    v, b, xs = (w.values.astype(np.float32), w.b.astype(np.float32), w.xstar.astype(np.float32))
+    k = 200
+    xo, _ = O.pcg(w.rowptr, w.colind, v[0], b[0], fixed_iters=k)
+    lo, _ = O.cg_adjoint(w.rowptr, w.colind, v[0], (xo - xs[0]).astype(np.float32), fixed_iters=k)
+    Go = O.grad_values(w.rowptr, w.colind, lo, xo)
+    x, lam, G, fi, ai = _pipeline(A, T(v), T(b), T(xs), fixed_iters=k)
+    assert H(fi.iters)[0] == k and H(ai.iters)[0] == k
     assert rel(H(x)[0], xo) < TOL_X32
+    assert rel(H(lam)[0], lo) < TOL_X32
+    assert rel(H(G)[0], Go) < TOL_X32
+    # the benchmark's fp32 run (tolerance 1e-8 on the recursive residual), at
+    # the GPU's own counts on the oracle's side
+    x, lam, G, fi, ai = _pipeline(A, T(v), T(b), T(xs), rtol=1e-8)
+    kf, ka = int(H(fi.iters)[0]), int(H(ai.iters)[0])
+    assert H(fi.status)[0] == L.SLA_CONVERGED and H(ai.status)[0] == L.SLA_CONVERGED
+    assert kf < 5000 and ka < 5000
+    xo, _ = O.pcg(w.rowptr, w.colind, v[0], b[0], fixed_iters=kf)
+    lo, _ = O.cg_adjoint(w.rowptr, w.colind, v[0], (xo - xs[0]).astype(np.float32), fixed_iters=ka)
+    Go = O.grad_values(w.rowptr, w.colind, lo, xo)
+    assert rel(H(x)[0], xo) < TOL_X32
+    assert rel(H(lam)[0], lo) < TOL_X32
+    assert rel(H(G)[0], Go) < TOL_X32
 
 
 def test_c4_batched_all_systems():
@@ -145,10 +187,17 @@ def test_c5_knn_fixed_and_tolerance(order):
     w = W.c5_knn(order=order)
     A = sla.CSR(T(w.rowptr), T(w.colind), symmetric=True)
     v, b, xs = w.values, w.b, w.xstar
-    k = 8
+    # forward, adjoint and value gradient element by element at a fixed count
+    k = 20
     xo, _ = O.pcg(w.rowptr, w.colind, v[0], b[0], fixed_iters=k)
-    x, fi = A.cg(T(v), T(b), fixed_iters=k)
+    lo, _ = O.cg_adjoint(w.rowptr, w.colind, v[0], xo - xs[0], fixed_iters=k)
+    Go = O.grad_values(w.rowptr, w.colind, lo, xo)
+    x, lam, G, fi, ai = _pipeline(A, T(v), T(b), T(xs), fixed_iters=k)
+    assert H(fi.iters)[0] == k and H(ai.iters)[0] == k
     assert rel(H(x)[0], xo) < TOL_X64
+    assert rel(H(lam)[0], lo) < TOL_G64
+    assert rel(H(G)[0], Go) < TOL_G64
+    # the benchmark's tolerance mode: properties at full size
     x, lam, G, fi, ai = _pipeline(A, T(v), T(b), T(xs), rtol=1e-8)
     assert H(fi.status)[0] == L.SLA_CONVERGED and H(ai.status)[0] == L.SLA_CONVERGED
     _properties(w, H(x)[0], H(lam)[0], H(G)[0], 1e-8, b[0], xs[0], v[0])

@@ -176,6 +176,38 @@ def _spmv_bound(rp, ci, v, x):
     return s
 
 
+def _skewed_csr(seed, n_rows, n_cols):
+    """Short rows (mean below the one-thread-a-row limit) with a 3000-entry row
+    every 997 rows: the 256-row chunks holding a long row exceed the staged
+    kernels' shared memory and walk their rows in global memory instead."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(1, 8, n_rows)
+    lens[::997] = 3000
+    rows = np.repeat(np.arange(n_rows, dtype=np.int64), lens)
+    cols = np.concatenate([np.sort(rng.choice(n_cols, k, replace=False)) for k in lens]).astype(np.int32)
+    rp = np.zeros(n_rows + 1, np.int32)
+    np.cumsum(np.bincount(rows, minlength=n_rows), out=rp[1:])
+    return rp, cols
+
+
+def test_spmv_and_gradients_on_skewed_short_rows():
+    """Chunks staged in shared memory and chunks too long for it, in one launch."""
+    n_rows, n_cols, B = 6000, 5000, 2
+    rp, ci = _skewed_csr(11, n_rows, n_cols)
+    A = make(rp, ci, B=B, symmetric=False, n_cols=n_cols)
+    assert A.props.lanes == 1
+    v = W.uniform(11, W.STREAM_WEIGHTS, B * ci.shape[0], -1, 1).reshape(B, -1)
+    x = W.uniform(11, W.STREAM_B, B * n_cols, -1, 1).reshape(B, n_cols)
+    y = H(A.spmv(T(v), T(x)))
+    y_o = O.spmv(rp, ci, v, x)
+    for s in range(B):
+        bound = _spmv_bound(rp, ci, v[s], x[s]) * 64 * np.finfo(np.float64).eps + 1e-300
+        assert np.all(np.abs(y[s] - y_o[s]) <= bound)
+    lam = W.uniform(12, W.STREAM_B, B * n_rows, -1, 1).reshape(B, n_rows)
+    assert np.array_equal(H(A.grad_values(T(lam), T(x))), O.grad_values(rp, ci, lam, x))
+    assert np.array_equal(H(A.matvec_grad_values(T(lam), T(x))), -O.grad_values(rp, ci, lam, x))
+
+
 @pytest.mark.parametrize("per_row", [5, 30, 60, 120, 250, 500])
 def test_spmv_parity_all_row_widths(per_row):
     n_rows, n_cols = 3001, 2503
@@ -233,6 +265,11 @@ def test_grad_values_bit_exact_on_same_inputs(dtype):
         gb = T(base).clone()
         A.grad_values(T(lam), T(x), out=gb, accumulate=True)
         assert np.array_equal(H(gb), O.grad_values(rp, ci, lam, x, grad=base))
+        # the matvec form gy_i x_j is the exact negation of -lambda_i x_j with lambda = gy
+        assert np.array_equal(H(A.matvec_grad_values(T(lam), T(x))), -O.grad_values(rp, ci, lam, x))
+        gb = T(base).clone()
+        A.matvec_grad_values(T(lam), T(x), out=gb, accumulate=True)
+        assert np.array_equal(H(gb), base - O.grad_values(rp, ci, lam, x))
 
 
 # ------------------------------------------------------------- PCG solves ----
@@ -252,18 +289,25 @@ def _cases():
 
 
 # (strategy, on-chip grid vectors, sliced short-row layout); on-chip "3" keeps
-# the vectors on chip but turns the two-barrier single-system form off
+# the vectors on chip but turns the two-barrier single-system form off; "2"
+# keeps only r and q on chip (x and M^-1 in HBM); sliced "u" is the sliced
+# layout with per-slice widths (uniform widths off), "n" without the rows of
+# irregular patterns sorted by length within 32-row windows
 SOLVER_VARIANTS = [
     (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"),
     (L.SLA_STRATEGY_GRID, "0", "1"), (L.SLA_STRATEGY_GRID, "1", "0"),
-    (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_BLOCK, "1", "1"),
-    (L.SLA_STRATEGY_CLUSTER, "1", "1")]
+    (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_GRID, "2", "1"),
+    (L.SLA_STRATEGY_GRID, "2", "0"), (L.SLA_STRATEGY_GRID, "1", "u"),
+    (L.SLA_STRATEGY_GRID, "0", "u"), (L.SLA_STRATEGY_GRID, "0", "n"),
+    (L.SLA_STRATEGY_BLOCK, "1", "1"), (L.SLA_STRATEGY_CLUSTER, "1", "1")]
 
 
 def _variant_env(monkeypatch, onchip, sell):
-    monkeypatch.setenv("SLA_GRID_ONCHIP", "0" if onchip == "0" else "1")
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip if onchip in ("0", "2") else "1")
     monkeypatch.setenv("SLA_GRID2", "0" if onchip == "3" else "1")
-    monkeypatch.setenv("SLA_SELL", sell)
+    monkeypatch.setenv("SLA_SELL", "0" if sell == "0" else "1")
+    monkeypatch.setenv("SLA_SELL_UNIFORM", "0" if sell == "u" else "1")
+    monkeypatch.setenv("SLA_SELL_SORT", "0" if sell == "n" else "1")
 
 
 @pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
@@ -287,6 +331,15 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
             assert A.props.grid_onchip in (0, 1)
         if strategy == L.SLA_STRATEGY_GRID and onchip == "1" and B == 1 and A.props.sliced:
             assert A.props.grid_onchip == 2, name
+        if strategy == L.SLA_STRATEGY_GRID and onchip == "2":
+            assert A.props.grid_onchip == 3 or A.props.lanes > 1, name
+        if sell == "u":
+            assert A.props.sliced in (0, 1, 3), name
+        if sell == "n":
+            assert A.props.sliced in (0, 1, 2), name
+        if name == "random3000" and strategy == L.SLA_STRATEGY_GRID and onchip in ("0", "2") \
+                and sell in ("1", "u"):
+            assert A.props.sliced == 3, name            # irregular rows: sorted windows
         for k in (1, 7, 60):
             x, info = A.cg(T(v.astype(npdt)), T(b.astype(npdt)), fixed_iters=k, strategy=strategy)
             xo, io = O.pcg(rp, ci, v.astype(npdt), b.astype(npdt), fixed_iters=k)
@@ -326,7 +379,7 @@ def test_grid_and_block_strategies_agree():
     assert np.all(np.abs(H(ig.iters) - H(ib.iters)) <= 2)
 
 
-@pytest.mark.parametrize("onchip", ["1", "0"])
+@pytest.mark.parametrize("onchip", ["1", "0", "2"])
 def test_results_are_bitwise_reproducible(onchip, monkeypatch):
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     w = W.c1_poisson64()
@@ -431,7 +484,7 @@ def test_adjoint_memory_does_not_grow_with_iterations():
 
 # ------------------------------------------------------------ edge cases ----
 
-@pytest.mark.parametrize("onchip", ["1", "3"])
+@pytest.mark.parametrize("onchip", ["1", "3", "2"])
 def test_edge_cases_match_oracle_outcomes(onchip, monkeypatch):
     _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.random_spd(300, 0.02, 4)
@@ -480,7 +533,7 @@ def test_single_unknown_and_empty_matrix():
     assert x.shape == (2, 0) and np.all(H(info.status) == 0) and np.all(H(info.iters) == 0)
 
 
-@pytest.mark.parametrize("onchip", ["1", "3", "0"])
+@pytest.mark.parametrize("onchip", ["1", "3", "0", "2"])
 def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
     _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.poisson2d(300)

@@ -9,6 +9,10 @@ call leaves in the shared array does not leak into the second.  This file is
 collected last so that a run stopping at the first failure has run every other
 test before it.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -82,3 +86,15 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     x = torch.empty(n, dtype=torch.float64, device=DEV)
     with pytest.raises(L.SlaError, match="built-in limit"):
         L.sla_cg_solve_noalloc(n, n, rp, ci, 1, L.SLA_F64, v, b, x, L.make_opts(), L.make_info())
+
+
+def test_noalloc_follows_the_current_context():
+    """A caller that manages its own contexts (the driver API's, or the device
+    after a reset) gets the scratch array of the context it calls from: in the
+    primary context, in two created contexts and back, two allocation-free
+    calls in a row match sla_cg_solve.  Runs as a separate process that makes
+    no PyTorch CUDA calls, so the contexts are the script's own."""
+    script = os.path.join(os.path.dirname(os.path.abspath(__file__)), "noalloc_contexts.py")
+    r = subprocess.run([sys.executable, script], capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "noalloc contexts: ok" in r.stdout
