@@ -59,7 +59,8 @@ class sla_csr_props(ctypes.Structure):
                 ("grid_tile_rows", ctypes.c_int32), ("sliced", ctypes.c_int32),
                 ("block_resident", ctypes.c_int32), ("cluster_fits", ctypes.c_int32),
                 ("n_items", ctypes.c_int32), ("item_rows_max", ctypes.c_int32),
-                ("item_smem_rows", ctypes.c_int32), ("interleaved", ctypes.c_int32)]
+                ("item_smem_rows", ctypes.c_int32), ("sliced_col_bytes", ctypes.c_int32),
+                ("interleaved", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p

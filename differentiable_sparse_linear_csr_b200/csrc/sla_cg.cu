@@ -76,8 +76,8 @@ struct CgArgs {
     int64_t sell_nnz;
     int sell_w;         // > 0: every slice of the sliced layout is sell_w entries wide
     const int32_t *sell_perm;   // or null: the row at each position of the sliced layout
-    int ldmode;         // sliced-matrix load mode of the HBM solver (see sell_load)
-    int l2_prefetch;    // HBM solver: row waves of the matrix stream prefetched into L2 ahead
+    const int16_t *sell_d16;    // or null: the sliced layout's columns as offsets from their row
+    int p_onchip;       // on-chip solver: the tile's own p also kept in shared memory
 };
 
 // ------------------------------------------------------------ helpers ----
@@ -273,33 +273,21 @@ __device__ void give_up(const CgArgs<T> &a) {
 }
 
 // ------------------------------------------------------- grid kernel ----
-constexpr int kMaxWaves = 128;   // row waves of one tile the L2 prefetch schedule covers
-
 // q = A p over rows [r0, r1) of the sliced layout with vectors in HBM, one row
-// a thread (rows r0 + tid, r0 + tid + NT, ...: "waves" of NT rows).  When
-// nwaves > 0, thread 0 keeps the matrix slots of the next D waves on their way
-// into L2 (bulk prefetch; wave_slot holds each wave's first slot).  Returns the
+// a thread; the matrix streams past L1 (no-allocate loads).  Returns the
 // thread's partial p.q.
-template <int MODE, int NT, typename T>
-__device__ __forceinline__ double sell_tile_hbm(const CgArgs<T> &a, const T *svals, const T *pg, T *q_out,
-                                                int q_off, int r0, int r1, const int *wave_slot, int nwaves) {
-    const int tid = threadIdx.x, D = a.l2_prefetch;
-    auto prefetch = [&](int w) {
-        const int b0 = wave_slot[w], b1 = wave_slot[w + 1];
-        if (b1 > b0) {
-            prefetch_l2_bulk(svals + b0, (unsigned)((b1 - b0) * sizeof(T)));
-            prefetch_l2_bulk(a.sell_cols + b0, (unsigned)((b1 - b0) * sizeof(int32_t)));
-        }
-    };
-    if (nwaves > 0 && tid == 0)
-        for (int w = 0; w < D && w < nwaves; ++w) prefetch(w);
+template <int NT, typename T>
+__device__ __forceinline__ double sell_tile_hbm(const CgArgs<T> &a, const T *svals, const T *pg, T *qg,
+                                                int r0, int r1) {
     double acc = 0.0;
-    int w = 0;
-    for (int i = r0 + tid; i < r1; i += NT, ++w) {
-        if (nwaves > 0 && tid == 0 && w + D < nwaves) prefetch(w + D);
-        const T qi = sell_row<MODE>(a.sell_ptr, a.sell_cols, svals, pg, i, a.n, a.sell_nnz, a.sell_w);
+    for (int i = r0 + threadIdx.x; i < r1; i += NT) {
         const int row = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i), a.n, kBndLocal) : i;
-        q_out[row - q_off] = qi;
+        const T qi = a.sell_d16
+                         ? sell_row<1, true>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, pg, i, row, a.n,
+                                             a.sell_nnz, a.sell_w)
+                         : sell_row<1, false>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, pg, i, row, a.n,
+                                              a.sell_nnz, a.sell_w);
+        qg[row] = qi;
         acc += (double)pg[row] * (double)qi;
     }
     return acc;
@@ -309,14 +297,11 @@ __device__ __forceinline__ double sell_tile_hbm(const CgArgs<T> &a, const T *sva
 // the whole solve and takes the decisions (breakdown, stop, alpha, beta) for
 // them itself from the shared partials; ONCHIP keeps x, r and M^-1 of its one
 // tile in shared memory and q in registers (RPT rows a thread), so only A and
-// p travel through L2/HBM each iteration.  RQS (vectors otherwise in HBM, one
-// tile a block) keeps r and q of the tile in shared memory: for systems whose
-// three on-chip vectors do not fit, it saves the r and q passes over HBM.
-template <typename T, int LANES, bool ONCHIP, int RPT, int NT, bool SELL, bool RQS = false>
-__global__ void __launch_bounds__(NT, (ONCHIP || RQS) ? 1 : 2)
+// p travel through L2/HBM each iteration.
+template <typename T, int LANES, bool ONCHIP, int RPT, int NT, bool SELL>
+__global__ void __launch_bounds__(NT, ONCHIP ? 1 : 2)
 cg_grid_kernel(CgArgs<T> a) {
-    static_assert(!(ONCHIP && RQS), "one on-chip layout at a time");
-    constexpr int LT = (ONCHIP || RQS) ? 1 : kMaxLocalTiles;   // tiles one block may own
+    constexpr int LT = ONCHIP ? 1 : kMaxLocalTiles;   // tiles one block may own
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ double red[4 * 33];
     __shared__ double l_rho[LT], l_nb[LT], l_rr[LT], l_alpha[LT];
@@ -341,28 +326,12 @@ cg_grid_kernel(CgArgs<T> a) {
     T *xs_ = reinterpret_cast<T *>(smem_raw);     // ONCHIP: [tile_rows] each
     T *rs_ = xs_ + (ONCHIP ? a.tile_rows : 0);
     T *ds_ = rs_ + (ONCHIP ? a.tile_rows : 0);
-    T *rq_ = reinterpret_cast<T *>(smem_raw);     // RQS: r [tile_rows], then q [tile_rows]
-    T *qq_ = rq_ + (RQS ? a.tile_rows : 0);
-    __shared__ int wave_slot[(SELL && !ONCHIP) ? kMaxWaves + 1 : 1];
-    int nwaves = 0;   // > 0: the SpMV prefetches its tile's matrix stream into L2
+    // ONCHIP with p_onchip: the tile's own rows of p, read by the p.q partials,
+    // x += alpha p and the direction update without a round trip to L2 (p is
+    // still written to global memory for the other tiles' gathers)
+    T *ps_ = (ONCHIP && a.p_onchip) ? ds_ + a.tile_rows : nullptr;
 
     if (blockIdx.x == 0 && tid == 0) a.sync[3] = (unsigned)a.B;
-    if constexpr (SELL && !ONCHIP) {
-        if (a.l2_prefetch > 0 && nlt == 1 && a.sell_rec == nullptr) {
-            const int tt = blockIdx.x % a.ntiles;
-            const int r0 = tt * a.tile_rows, r1 = min(n, r0 + a.tile_rows);
-            const int nw = (r1 - r0 + NT - 1) / NT;
-            if (nw <= kMaxWaves) {
-                // wave w covers rows [r0 + w NT, min(r1, r0 + (w+1) NT)): its slots start at
-                // the slice holding its first row; the table ends at the slice after r1 - 1
-                for (int w = tid; w <= nw; w += NT) {
-                    const int sl = w < nw ? (r0 + w * NT) / kSellRows : (r1 + kSellRows - 1) / kSellRows;
-                    wave_slot[w] = __ldg(a.sell_ptr + sl);
-                }
-                nwaves = nw;
-            }
-        }
-    }
 
     // ---- init: r = b - A x0 (or b), z = M^-1 r, p = z; partials of b.b, r.z, r.r
     for (int lt = 0; lt < nlt; ++lt) {
@@ -394,13 +363,13 @@ cg_grid_kernel(CgArgs<T> a) {
             const T zi = di * ri;
             pg[i] = zi;
             if constexpr (ONCHIP) {
+                if (ps_) ps_[i - r0] = zi;
                 xs_[i - r0] = xi;
                 rs_[i - r0] = ri;
                 ds_[i - r0] = di;
             } else {
                 if (!a.x0_given) xg[i] = T(0);
-                if constexpr (RQS) rq_[i - r0] = ri;
-                else a.r[(int64_t)s * n + i] = ri;
+                a.r[(int64_t)s * n + i] = ri;
                 a.d[(int64_t)s * n + i] = di;
             }
             acc[0] += (double)bi * (double)bi;
@@ -488,7 +457,7 @@ cg_grid_kernel(CgArgs<T> a) {
                         if (i < r1) {
                             const T qi = sell_row_rec<false>(a.sell_ptr, rec, pg, i, n, a.sell_nnz);
                             qreg[j] = qi;
-                            acc[0] += (double)pg[i] * (double)qi;
+                            acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
                         }
                     }
                 } else {
@@ -497,9 +466,13 @@ cg_grid_kernel(CgArgs<T> a) {
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
                         if (i < r1) {
-                            const T qi = sell_row<false>(a.sell_ptr, a.sell_cols, svals, pg, i, n, a.sell_nnz, a.sell_w);
+                            const T qi = a.sell_d16
+                                ? sell_row<0, true>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, pg, i, i, n,
+                                                    a.sell_nnz, a.sell_w)
+                                : sell_row<0, false>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, pg, i, i, n,
+                                                     a.sell_nnz, a.sell_w);
                             qreg[j] = qi;
-                            acc[0] += (double)pg[i] * (double)qi;
+                            acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
                         }
                     }
                 }
@@ -510,36 +483,29 @@ cg_grid_kernel(CgArgs<T> a) {
                     if (i < r1) {
                         const T qi = row_dot<T, 1>(a.rowptr, a.colind, vs, pg, i, 0, n, a.nnz);
                         qreg[j] = qi;
-                        acc[0] += (double)pg[i] * (double)qi;
+                        acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
                     }
                 }
             } else if constexpr (SELL) {
-                T *qg = RQS ? qq_ : a.q + (int64_t)s * n;   // q of row i at qg[i - qoff]
-                const int qoff = RQS ? r0 : 0;
+                T *qg = a.q + (int64_t)s * n;
                 if (a.sell_rec) {
                     const SellRec<T> *rec = a.sell_rec + (int64_t)s * a.sell_nnz;
                     for (int i = r0 + tid; i < r1; i += NT) {
                         const T qi = sell_row_rec<true>(a.sell_ptr, rec, pg, i, n, a.sell_nnz);
                         const int row = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i), n, kBndLocal) : i;
-                        qg[row - qoff] = qi;
+                        qg[row] = qi;
                         acc[0] += (double)pg[row] * (double)qi;
                     }
                 } else {
                     const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
-                    switch (a.ldmode) {
-                        case 0: acc[0] = sell_tile_hbm<0, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
-                        case 2: acc[0] = sell_tile_hbm<2, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
-                        case 3: acc[0] = sell_tile_hbm<3, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
-                        default: acc[0] = sell_tile_hbm<1, NT>(a, svals, pg, qg, qoff, r0, r1, wave_slot, nwaves); break;
-                    }
+                    acc[0] = sell_tile_hbm<NT>(a, svals, pg, qg, r0, r1);
                 }
             } else {
-                T *qg = RQS ? qq_ : a.q + (int64_t)s * n;   // q of row i at qg[i - qoff]
-                const int qoff = RQS ? r0 : 0;
+                T *qg = a.q + (int64_t)s * n;
                 for (int i = r0 + sub; i < r1; i += NSUB) {
                     const T qi = row_dot<T, LANES>(a.rowptr, a.colind, vs, pg, i, lane, n, a.nnz);
                     if (lane == 0) {
-                        qg[i - qoff] = qi;
+                        qg[i] = qi;
                         acc[0] += (double)pg[i] * (double)qi;
                     }
                 }
@@ -585,14 +551,12 @@ cg_grid_kernel(CgArgs<T> a) {
                     }
                 }
             } else {
-                // r and q of row i at rg[i - off], qg[i - off]
-                T *rg = RQS ? rq_ : a.r + (int64_t)s * n;
-                const T *qg = RQS ? qq_ : a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
-                const int off = RQS ? r0 : 0;
+                T *rg = a.r + (int64_t)s * n;
+                const T *qg = a.q + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
 #pragma unroll 4
                 for (int i = r0 + tid; i < r1; i += NT) {
-                    const T ri = rg[i - off] - al * qg[i - off];
-                    rg[i - off] = ri;
+                    const T ri = rg[i] - al * qg[i];
+                    rg[i] = ri;
                     const T zi = dg[i] * ri;
                     acc[0] += (double)ri * (double)zi;
                     acc[1] += (double)ri * (double)ri;
@@ -619,7 +583,7 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                 for (int j = 0; j < RPT; ++j) {
                     const int i = r0 + tid + j * NT;
-                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * pg[i];
+                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * (ps_ ? ps_[i - r0] : pg[i]);
                 }
             } else {
                 T *xg = a.x + (int64_t)s * n;
@@ -654,13 +618,16 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
-                        if (i < r1) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pg[i];
+                        if (i < r1) {
+                            const T pn = ds_[i - r0] * rs_[i - r0] + bt * (ps_ ? ps_[i - r0] : pg[i]);
+                            pg[i] = pn;
+                            if (ps_) ps_[i - r0] = pn;
+                        }
                     }
                 } else {
-                    const T *rg = RQS ? rq_ : a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
-                    const int off = RQS ? r0 : 0;
+                    const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
 #pragma unroll 4
-                    for (int i = r0 + tid; i < r1; i += NT) pg[i] = dg[i] * rg[i - off] + bt * pg[i];
+                    for (int i = r0 + tid; i < r1; i += NT) pg[i] = dg[i] * rg[i] + bt * pg[i];
                 }
             }
             __syncthreads();
@@ -801,7 +768,11 @@ cg_grid2_kernel(CgArgs<T> a) {
         for (int j = 0; j < RPT; ++j) {
             const int i = r0 + tid + j * NT;
             if (i < r1) {
-                const T qi = sell_row_dir<T>(a.sell_ptr, a.sell_cols, svals, zg, pprev, bt, i, a.n, a.sell_nnz, a.sell_w);
+                const T qi = a.sell_d16
+                    ? sell_row_dir<true>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, zg, pprev, bt, i, a.n,
+                                         a.sell_nnz, a.sell_w)
+                    : sell_row_dir<false>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, zg, pprev, bt, i, a.n,
+                                          a.sell_nnz, a.sell_w);
                 qreg[j] = qi;
                 T pi;
                 if constexpr (sizeof(T) == 8) pi = __fma_rn(bt, pprev[i], __dmul_rn(ds[i - r0], rs[i - r0]));
@@ -1742,10 +1713,6 @@ template <typename T, int RPT, bool SELL>
 static const void *onchip_fn() {
     return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, true, RPT, kOnchipThreads, SELL>);
 }
-template <typename T, bool SELL>
-static const void *rqs_fn() {
-    return reinterpret_cast<const void *>(&cg_grid_kernel<T, 1, false, 1, kOnchipThreads, SELL, true>);
-}
 template <typename T, int RPT>
 static const void *grid2_fn() {
     return reinterpret_cast<const void *>(&cg_grid2_kernel<T, RPT, kOnchipThreads>);
@@ -1804,14 +1771,8 @@ static const void *pick_il(sla_dtype dt, int B) {
                   : reinterpret_cast<const void *>(&cg_grid_il_kernel<float, 4>);
 }
 
-static const void *pick_rqs(sla_dtype dt, bool sell) {
-    if (dt == SLA_F64) return sell ? rqs_fn<double, true>() : rqs_fn<double, false>();
-    return sell ? rqs_fn<float, true>() : rqs_fn<float, false>();
-}
-
 static const void *pick_grid(const Csr *h, bool sell) {
     if (h->onchip) return pick_onchip(h->dtype, h->onchip_rpt, sell);
-    if (h->rqs) return pick_rqs(h->dtype, sell);
     if (sell) return h->dtype == SLA_F64 ? grid_sell_fn<double>() : grid_sell_fn<float>();
     return pick_fn(true, h->dtype, h->lanes);
 }
@@ -1872,9 +1833,8 @@ sla_status cg_configure(Csr *h) {
     // On-chip variant: one 1024-thread block per SM, x, r, M^-1 of the block's
     // rows in shared memory, at most 16 rows a thread.
     h->onchip = false;
-    // SLA_GRID_ONCHIP=0: vectors in HBM; =2: only the r-and-q variant below
     const char *oc = getenv("SLA_GRID_ONCHIP");
-    if (h->lanes == 1 && n > 0 && !(oc && (oc[0] == '0' || oc[0] == '2'))) {
+    if (h->lanes == 1 && n > 0 && !(oc && oc[0] == '0')) {
         int32_t tr = 0, nt = 0;
         layout(h, h->num_sms, &tr, &nt);
         const int rpt = (tr + kOnchipThreads - 1) / kOnchipThreads;
@@ -1884,7 +1844,7 @@ sla_status cg_configure(Csr *h) {
             for (int sv = 0; sv < 3; ++sv)
                 SLA_CHECK_CUDA(cudaFuncSetAttribute(
                     sv < 2 ? pick_onchip(h->dtype, rpt, sv != 0) : pick_grid2(h->dtype, rpt),
-                    cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 16384));
+                    cudaFuncAttributeMaxDynamicSharedMemorySize, sv < 2 ? optin - 4096 : optin - 16384));
             const void *f = pick_onchip(h->dtype, rpt, true);
             int per_sm = 0;
             SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kOnchipThreads, smem));
@@ -1910,38 +1870,23 @@ sla_status cg_configure(Csr *h) {
                 const bool l1_fits = smem + 2 * (size_t)tr * ts <= (size_t)smem_sm;
                 h->grid2 = h->batch == 1 && nt <= h->num_sms && per_sm2 >= 1 &&
                            (l1_fits || (g2 && g2[0] == '2')) && !(g2 && g2[0] == '0');
+                // The three-barrier solver also keeps the tile's own p on chip when a
+                // fourth vector fits (SLA_GRID_P4=0 turns it off).
+                const char *p4 = getenv("SLA_GRID_P4");
+                h->p_onchip = false;
+                if (!h->grid2 && 4 * (size_t)tr * ts + 4096 <= (size_t)optin && !(p4 && p4[0] == '0')) {
+                    int per_sm4 = 0;
+                    SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                        &per_sm4, f, kOnchipThreads, 4 * (size_t)tr * ts));
+                    if (per_sm4 >= 1) {
+                        h->p_onchip = true;
+                        h->grid_smem = 4 * (size_t)tr * ts;
+                    }
+                }
             }
         }
     }
-    // Vectors in HBM except r and q, which stay in shared memory: one 1024-thread
-    // block per SM whose tile's r and q fit (systems too large for the on-chip
-    // variant's three vectors, e.g. 2 M fp64 rows).  SLA_GRID_RQS=0 turns it off.
-    h->rqs = false;
-    const char *rq = getenv("SLA_GRID_RQS");
-    if (!h->onchip && h->lanes == 1 && n > 0 && !(oc && oc[0] == '0') && !(rq && rq[0] == '0')) {
-        int32_t tr = 0, nt = 0;
-        layout(h, h->num_sms, &tr, &nt);
-        const size_t smem = 2 * (size_t)tr * ts;
-        if ((int64_t)h->batch * nt <= h->num_sms && smem + 4096 <= (size_t)optin) {
-            for (int sv = 0; sv < 2; ++sv)
-                SLA_CHECK_CUDA(cudaFuncSetAttribute(pick_rqs(h->dtype, sv != 0),
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    optin - 4096));
-            int per_sm = 0;
-            SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                &per_sm, pick_rqs(h->dtype, true), kOnchipThreads, smem));
-            if (per_sm >= 1) {
-                h->rqs = true;
-                h->grid_smem = smem;
-                h->grid_threads = kOnchipThreads;
-                h->grid_blocks = h->num_sms;
-                h->tile_rows = tr;
-                h->ntiles = nt;
-                h->il_blocks = 0;
-            }
-        }
-    }
-    if (!h->onchip && !h->rqs) {
+    if (!h->onchip) {
         int per_sm = 0;
         SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
             &per_sm, pick_fn(true, h->dtype, h->lanes), kCgThreads, 0));
@@ -2156,10 +2101,7 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
     a.timeout_ns = o->wait_timeout_ns > 0 ? o->wait_timeout_ns : kDefaultTimeoutNs;
     a.tile_rows = h->tile_rows;
     a.ntiles = h->ntiles;
-    a.ldmode = 1;
-    if (const char *e = getenv("SLA_LDMODE")) a.ldmode = atoi(e);
-    a.l2_prefetch = 0;
-    if (const char *e = getenv("SLA_L2_PREFETCH")) a.l2_prefetch = atoi(e);
+    a.p_onchip = h->p_onchip ? 1 : 0;
     if (h->dep_lo != nullptr && pattern_is_forward_or_sym(h, rowptr)) {
         a.dep_lo = h->dep_lo;
         a.dep_hi = h->dep_hi;
@@ -2252,6 +2194,7 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             a.sell_nnz = h->sell_nnz;
             a.sell_w = h->sell_w;
             a.sell_perm = h->sell_perm;
+            a.sell_d16 = h->sell_d16;
             const char *pk = getenv("SLA_SELL_PACK");
             const bool pack = pk && pk[0] == '1' && !(h->grid2 && a.B == 1);
             if (pack) {

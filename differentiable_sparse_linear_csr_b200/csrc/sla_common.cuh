@@ -108,7 +108,7 @@ struct Csr {
     bool onchip = false;               // grid solver keeps x, r, M^-1 in shared memory
     int32_t onchip_rpt = 0;            // rows a thread in the on-chip grid solver
     bool grid2 = false;                // single system, on chip, sliced: two barriers an iteration
-    bool rqs = false;                  // grid solver keeps r and q in shared memory (x, M^-1 in HBM)
+    bool p_onchip = false;             // on-chip solver keeps the tile's own p in shared memory too
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block
@@ -137,6 +137,7 @@ struct Csr {
     int32_t sell_w = 0;                // > 0: every slice padded to this width (no offsets needed)
     int32_t *sell_perm = nullptr;      // owned [n_rows] or null: row at each position (rows of each
                                        // 32-row window ordered by decreasing length)
+    int16_t *sell_d16 = nullptr;       // owned [sell_nnz] or null: columns as offsets from their row
     int32_t *sell_ptr = nullptr;       // owned [n_slices + 1]: first entry of each slice
     int32_t *sell_cols = nullptr;      // owned [sell_nnz]: column (own row for padding)
     int32_t *sell_map = nullptr;       // owned [sell_nnz]: CSR position, -1 for padding
@@ -169,7 +170,7 @@ sla_status exclusive_scan(const unsigned *in, unsigned *out, int64_t n, void *ws
 constexpr int kSellRows = 8;
 constexpr int kSellSortWindow = 32;   // rows sorted by length together (one warp's rows)
 // sort_ok: the solver that uses this layout keeps q by row index (vectors in
-// HBM or r and q in shared memory), so rows may be permuted within windows.
+// HBM), so rows may be permuted within windows.
 sla_status build_sell(Csr *h, bool sort_ok, cudaStream_t s);
 sla_status cg_tile_deps(Csr *h, cudaStream_t s);   // in sla_cg.cu
 // vals_sell[b][slot] = vals[b][sell_map[slot]] (0 for padding), every system.

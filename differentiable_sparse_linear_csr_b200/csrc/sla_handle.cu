@@ -436,8 +436,8 @@ sla_status create_handle(int32_t n_rows, int32_t n_cols, int64_t nnz, const int3
         if (st != SLA_OK) return fail(st);
         const char *sv = getenv("SLA_SELL");
         if (h->lanes == 1 && n_rows > 0 && !(sv && sv[0] == '0')) {
-            // rows sorted within windows only for solver variants that keep q by row and
-            // whose windows never straddle a tile (the interleaved batch solver does not)
+            // rows sorted within windows only for the solver variant that keeps q in
+            // HBM by row, with windows inside tiles (not the interleaved batch solver)
             const bool sort_ok = !h->onchip && h->il_blocks == 0 && h->tile_rows % kSellSortWindow == 0;
             st = build_sell(h, sort_ok, s);
             if (st != SLA_OK) return fail(st);
@@ -464,6 +464,7 @@ extern "C" sla_status sla_csr_destroy(sla_csr_t hh) {
     cudaFree(h->sell_cols);
     cudaFree(h->sell_map);
     cudaFree(h->sell_perm);
+    cudaFree(h->sell_d16);
     cudaFree(h->dep_lo);
     cudaFree(h->dep_hi);
     cudaFree(h->seg);
@@ -488,9 +489,10 @@ extern "C" sla_status sla_csr_get_props(sla_csr_t hh, sla_csr_props *p) {
     p->grid_blocks = h->grid_blocks;
     p->block_fits = h->block_fits ? 1 : 0;
     p->has_transpose = h->has_transpose ? 1 : 0;
-    p->grid_onchip = h->onchip ? (h->grid2 && h->has_sell ? 2 : 1) : (h->rqs ? 3 : 0);
+    p->grid_onchip = h->onchip ? (h->grid2 && h->has_sell ? 2 : 1) : 0;
     p->grid_tile_rows = h->tile_rows;
     p->sliced = h->has_sell ? (h->sell_w > 0 ? 2 : (h->sell_perm ? 3 : 1)) : 0;
+    p->sliced_col_bytes = h->has_sell ? (h->sell_d16 ? 2 : 4) : 0;
     p->block_resident = h->block_mres ? 1 : 0;
     p->cluster_fits = h->cluster_fits ? 1 : 0;
     p->n_items = h->n_items;

@@ -88,21 +88,13 @@ __device__ __forceinline__ T row_dot_perm(const int32_t *__restrict__ rowptr,
     return s;
 }
 
-// Loads of the sliced layout's entries, by MODE:
-//   0  the default allocating read-only load (the matrix stays in L2 and L1);
-//   1  ld.global.nc.L1::no_allocate: in the solver whose vectors live in HBM the
-//      matrix streams through once per iteration and L1 is better left to the
-//      gathered vector; where the matrix stays in L2 the allocating load is
-//      faster (a slice step uses half a 128-byte line, the next step the other);
-//   2  as 1, with an L2 evict-first policy, so that the streamed matrix leaves
-//      L2 before the vectors;
-//   3  as 1, asking L2 to fetch the whole 256-byte block on a miss.
-__device__ __forceinline__ unsigned long long l2_evict_first_policy() {
-    unsigned long long pol;
-    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
+// Loads of the sliced layout's entries: MODE 0 is the default allocating
+// read-only load (where the matrix stays in L2, a slice step uses half a
+// 128-byte line and the next step the other half); MODE 1 is
+// ld.global.nc.L1::no_allocate, for the solver whose vectors live in HBM: the
+// matrix streams through once per iteration and L1 is better left to the
+// gathered vector.  (L2 evict-first and 256-byte prefetch-size hints, and a
+// bulk L2 prefetch of the tile's next rows, measured no faster.)
 template <int MODE, typename T>
 __device__ __forceinline__ T sell_load(const T *p) {
     static_assert(sizeof(T) == 4 || sizeof(T) == 8, "4- or 8-byte entries");
@@ -110,42 +102,29 @@ __device__ __forceinline__ T sell_load(const T *p) {
         return __ldg(p);
     } else if constexpr (sizeof(T) == 8) {
         double v;
-        if constexpr (MODE == 1)
-            asm volatile("ld.global.nc.L1::no_allocate.f64 %0, [%1];" : "=d"(v) : "l"(p));
-        else if constexpr (MODE == 2)
-            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f64 %0, [%1], %2;"
-                         : "=d"(v) : "l"(p), "l"(l2_evict_first_policy()));
-        else
-            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.f64 %0, [%1];" : "=d"(v) : "l"(p));
+        asm volatile("ld.global.nc.L1::no_allocate.f64 %0, [%1];" : "=d"(v) : "l"(p));
         return (T)v;
     } else if constexpr (std::is_same<T, float>::value) {
         float v;
-        if constexpr (MODE == 1)
-            asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
-        else if constexpr (MODE == 2)
-            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;"
-                         : "=f"(v) : "l"(p), "l"(l2_evict_first_policy()));
-        else
-            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.f32 %0, [%1];" : "=f"(v) : "l"(p));
+        asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
         return v;
     } else {
         int v;
-        if constexpr (MODE == 1)
-            asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
-        else if constexpr (MODE == 2)
-            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.s32 %0, [%1], %2;"
-                         : "=r"(v) : "l"(p), "l"(l2_evict_first_policy()));
-        else
-            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.s32 %0, [%1];" : "=r"(v) : "l"(p));
+        asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];" : "=r"(v) : "l"(p));
         return (T)v;
     }
 }
 
-// Asks L2 to fetch [p, p + bytes) from memory ahead of use (a bulk prefetch
-// issued by one thread; no registers or shared memory wait for it).  p must be
-// 16-byte aligned and bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, unsigned bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+// A column stored as a 16-bit offset from its row (the sliced layout's
+// compact columns), loaded like sell_load's MODE and sign-extended.
+template <int MODE>
+__device__ __forceinline__ int sell_load_d16(const int16_t *p) {
+    short v;
+    if constexpr (MODE == 0)
+        v = __ldg(p);
+    else
+        asm volatile("ld.global.nc.L1::no_allocate.s16 %0, [%1];" : "=h"(v) : "l"(p));
+    return (int)v;
 }
 
 // First slot and width of row i's slice: computed when every slice has the
@@ -170,18 +149,21 @@ __device__ __forceinline__ void sell_slice(const int32_t *__restrict__ sptr, int
 // interleaving a thread's rows spreads its gathers of v and measured slower,
 // and so did loading a row's entries into registers before gathering (the
 // registers spill at the solver's 64-register budget).  uw > 0: every slice is
-// uw wide (no slice offsets read).
-template <int STREAM, typename T>
+// uw wide (no slice offsets read).  i is the row's position in the layout and
+// row the row itself (they differ when windows are sorted); with D16 the
+// columns come from d16 as offsets from row, else from cols.
+template <int STREAM, bool D16, typename T>
 __device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
-                                      const int32_t *__restrict__ cols,
-                                      const T *__restrict__ vals, const T *v, int i,
+                                      const int32_t *__restrict__ cols, const int16_t *__restrict__ d16,
+                                      const T *__restrict__ vals, const T *v, int i, int row,
                                       int ncols, int64_t nslots, int uw) {
     int base, w;
     sell_slice(sptr, i, uw, base, w);
     T s = T(0);
     for (int k = 0; k < w; ++k) {
         const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
-        s += sell_load<STREAM>(vals + t) * v[SLA_IDX(sell_load<STREAM>(cols + t), ncols, kBndColumn)];
+        const int c = D16 ? row + sell_load_d16<STREAM>(d16 + t) : sell_load<STREAM>(cols + t);
+        s += sell_load<STREAM>(vals + t) * v[SLA_IDX(c, ncols, kBndColumn)];
     }
     return s;
 }
@@ -235,9 +217,9 @@ __device__ __forceinline__ T sell_row_rec(const int32_t *__restrict__ sptr, cons
 // Row of the sliced layout times the direction p_k = z + beta p_prev, formed
 // per gathered entry with one fused multiply-add (the owner of each row forms
 // the same value the same way from its own M^-1 r, rounded once, as z).
-template <typename T>
+template <bool D16, typename T>
 __device__ __forceinline__ T sell_row_dir(const int32_t *__restrict__ sptr,
-                                          const int32_t *__restrict__ cols,
+                                          const int32_t *__restrict__ cols, const int16_t *__restrict__ d16,
                                           const T *__restrict__ vals, const T *z, const T *pprev,
                                           T beta, int i, int ncols, int64_t nslots, int uw) {
     int base, w;
@@ -245,7 +227,7 @@ __device__ __forceinline__ T sell_row_dir(const int32_t *__restrict__ sptr,
     T s = T(0);
     for (int k = 0; k < w; ++k) {
         const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
-        const int c = SLA_IDX(__ldg(cols + t), ncols, kBndColumn);
+        const int c = SLA_IDX(D16 ? i + sell_load_d16<0>(d16 + t) : __ldg(cols + t), ncols, kBndColumn);
         T pj;
         if constexpr (sizeof(T) == 8) pj = __fma_rn(beta, pprev[c], z[c]);
         else pj = __fmaf_rn(beta, pprev[c], z[c]);

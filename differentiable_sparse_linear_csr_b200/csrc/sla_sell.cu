@@ -20,7 +20,12 @@
 //    and the padding shrinks (a 10-entry-mean kNN graph: 19 % -> 6 %).  A
 //    window is one warp's rows in the solver, so each warp still handles the
 //    same rows; sell_perm maps a position to its row.  Each row's entries keep
-//    their stored order, so its sum is unchanged.
+//    their stored order, so its sum is unchanged;
+//  - compact columns: when every |column - row| < 2^15 (stencils, grids,
+//    bandwidth-reduced orderings), the columns are also kept as 16-bit offsets
+//    from their row (sell_d16), which the solver reads instead: 2 bytes an
+//    entry instead of 4 in the matrix stream.
+#include <climits>
 #include <cstdlib>
 
 #include "sla_common.cuh"
@@ -61,29 +66,50 @@ __global__ void sell_width_kernel(int n, const int32_t *__restrict__ rowptr, con
     cnt[sl] = (unsigned)(w * kSellRows);
 }
 
+// Columns, slot-to-entry map and 16-bit column offsets (clamped; *dmax
+// receives the largest |column - row| so the caller can tell whether they hold).
 __global__ void sell_fill_kernel(int n, const int32_t *__restrict__ rowptr,
                                  const int32_t *__restrict__ colind, const int32_t *__restrict__ sptr,
                                  const int32_t *__restrict__ perm, int32_t *__restrict__ cols,
-                                 int32_t *__restrict__ map) {
+                                 int32_t *__restrict__ map, int16_t *__restrict__ d16, int *__restrict__ dmax) {
     const int64_t sl = blockIdx.x * (int64_t)(blockDim.x / kSellRows) + threadIdx.x / kSellRows;
     const int l = threadIdx.x % kSellRows;
     const int64_t nsl = ((int64_t)n + kSellRows - 1) / kSellRows;
-    if (sl >= nsl) return;
-    const int64_t i = sl * kSellRows + l;
-    const int base = sptr[sl], w = (sptr[sl + 1] - base) / kSellRows;
-    const int row = i < n ? (perm ? perm[i] : (int)i) : 0;
-    const int t0 = i < n ? rowptr[row] : 0, len = i < n ? rowptr[row + 1] - t0 : 0;
-    const int own = row;
-    for (int k = 0; k < w; ++k) {
-        const int slot = base + k * kSellRows + l;
-        if (k < len) {
-            cols[slot] = colind[t0 + k];
-            map[slot] = t0 + k;
-        } else {
-            cols[slot] = own;
-            map[slot] = -1;
+    int far = 0;
+    if (sl < nsl) {
+        const int64_t i = sl * kSellRows + l;
+        const int base = sptr[sl], w = (sptr[sl + 1] - base) / kSellRows;
+        const int row = i < n ? (perm ? perm[i] : (int)i) : 0;
+        const int t0 = i < n ? rowptr[row] : 0, len = i < n ? rowptr[row + 1] - t0 : 0;
+        for (int k = 0; k < w; ++k) {
+            const int slot = base + k * kSellRows + l;
+            const int c = k < len ? colind[t0 + k] : row;
+            cols[slot] = c;
+            map[slot] = k < len ? t0 + k : -1;
+            const long long d = (long long)c - row;
+            const long long ad = d < 0 ? -d : d;
+            far = (int)max((long long)far, ad < INT_MAX ? ad : (long long)INT_MAX);
+            d16[slot] = (int16_t)(d < -32768 ? -32768 : (d > 32767 ? 32767 : d));
         }
     }
+    for (int o = 16; o > 0; o >>= 1) far = max(far, __shfl_xor_sync(0xffffffffu, far, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(dmax, far);
+}
+
+// Keeps the 16-bit column offsets when every |column - row| fits (stencils and
+// bandwidth-reduced orderings): 2 bytes an entry instead of 4 in the matrix
+// stream.  SLA_SELL_D16=0 turns them off.
+static sla_status finish_d16(Csr *h, int *dmax_dev, cudaStream_t s) {
+    int dmax = INT_MAX;
+    SLA_CHECK_CUDA(cudaMemcpyAsync(&dmax, dmax_dev, sizeof dmax, cudaMemcpyDeviceToHost, s));
+    SLA_CHECK_CUDA(cudaStreamSynchronize(s));
+    cudaFree(dmax_dev);
+    const char *e = getenv("SLA_SELL_D16");
+    if (dmax > 32767 || (e && e[0] == '0')) {
+        cudaFree(h->sell_d16);
+        h->sell_d16 = nullptr;
+    }
+    return SLA_OK;
 }
 
 template <typename T>
@@ -119,16 +145,20 @@ sla_status build_sell(Csr *h, bool sort_ok, cudaStream_t s) {
         h->sell_nnz = uslots;
         SLA_CHECK_CUDA(cudaMalloc(&h->sell_cols, (size_t)uslots * sizeof(int32_t)));
         SLA_CHECK_CUDA(cudaMalloc(&h->sell_map, (size_t)uslots * sizeof(int32_t)));
+        SLA_CHECK_CUDA(cudaMalloc(&h->sell_d16, (size_t)uslots * sizeof(int16_t)));
+        int *dmax = nullptr;
+        SLA_CHECK_CUDA(cudaMalloc(&dmax, sizeof(int)));
+        SLA_CHECK_CUDA(cudaMemsetAsync(dmax, 0, sizeof(int), s));
         constexpr int kThreads = 256;
         const unsigned grid = (unsigned)((nsl + kThreads / kSellRows - 1) / (kThreads / kSellRows));
         sell_fill_kernel<<<grid, kThreads, 0, s>>>(n, h->rowptr, h->colind, h->sell_ptr, nullptr,
-                                                   h->sell_cols, h->sell_map);
+                                                   h->sell_cols, h->sell_map, h->sell_d16, dmax);
         SLA_CHECK_LAUNCH();
         h->has_sell = true;
-        return SLA_OK;
+        return finish_d16(h, dmax, s);
     }
     // Irregular rows: sort each 32-row window by length when the solver keeps q
-    // by row index (SLA_SELL_SORT=0 turns it off).
+    // in HBM by row index (SLA_SELL_SORT=0 turns it off).
     const char *se = getenv("SLA_SELL_SORT");
     if (sort_ok && h->row_min != h->row_max && !(se && se[0] == '0')) {
         SLA_CHECK_CUDA(cudaMalloc(&h->sell_perm, (size_t)n * sizeof(int32_t)));
@@ -164,13 +194,17 @@ sla_status build_sell(Csr *h, bool sort_ok, cudaStream_t s) {
     const size_t z = (size_t)(total > 0 ? total : 1);
     SLA_CHECK_CUDA(cudaMalloc(&h->sell_cols, z * sizeof(int32_t)));
     SLA_CHECK_CUDA(cudaMalloc(&h->sell_map, z * sizeof(int32_t)));
+    SLA_CHECK_CUDA(cudaMalloc(&h->sell_d16, z * sizeof(int16_t)));
+    int *dmax = nullptr;
+    SLA_CHECK_CUDA(cudaMalloc(&dmax, sizeof(int)));
+    SLA_CHECK_CUDA(cudaMemsetAsync(dmax, 0, sizeof(int), s));
     constexpr int kThreads = 256;
     const unsigned grid = (unsigned)((nsl + kThreads / kSellRows - 1) / (kThreads / kSellRows));
     sell_fill_kernel<<<grid, kThreads, 0, s>>>(n, h->rowptr, h->colind, h->sell_ptr, h->sell_perm,
-                                               h->sell_cols, h->sell_map);
+                                               h->sell_cols, h->sell_map, h->sell_d16, dmax);
     SLA_CHECK_LAUNCH();
     h->has_sell = true;
-    return SLA_OK;
+    return finish_d16(h, dmax, s);
 }
 
 sla_status sell_values(const Csr *h, const void *vals, void *vals_sell, cudaStream_t s) {

@@ -66,16 +66,20 @@ spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32
     const int e0 = __ldg(rowptr + r0), e1 = __ldg(rowptr + r1);
     const int t0 = i < r1 ? __ldg(rowptr + i) : 0, t1 = i < r1 ? __ldg(rowptr + i + 1) : 0;
     const bool staged = e1 - e0 <= cap;
-    if (staged)
+    if (staged) {
+#pragma unroll 4
         for (int t = e0 + tid; t < e1; t += kChunkRows)
             s_cols[t - e0] = __ldg(colind + SLA_IDX(t, nnz, kBndEntry));
+    }
     for (int sys = blockIdx.y; sys < B; sys += gridDim.y) {
         const T *vb = vals + (int64_t)sys * nnz;
         const T *xb = x + (int64_t)sys * x_stride;
         T s = T(0);
         if (staged) {
+#pragma unroll 4
             for (int t = e0 + tid; t < e1; t += kChunkRows) s_vals[t - e0] = __ldg(vb + SLA_IDX(t, nnz, kBndEntry));
             __syncthreads();
+#pragma unroll 4
             for (int t = t0; t < t1; ++t)
                 s += s_vals[t - e0] * __ldg(xb + SLA_IDX(s_cols[t - e0], x_stride, kBndColumn));
             __syncthreads();
@@ -142,6 +146,7 @@ grad_staged_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__
         const T *xb = x + (int64_t)sys * n_cols;
         T *gb = grad + (int64_t)sys * nnz;
         if (staged) {
+#pragma unroll 4
             for (int t = e0 + tid; t < e1; t += kChunkRows) {
                 const int tt = SLA_IDX(t, nnz, kBndEntry);
                 const T p = __ldg(lb + s_row[t - e0]) * __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn));

@@ -129,11 +129,8 @@ typedef struct {
     int32_t grid_onchip;      /* 1 if the grid solver keeps x, r, M^-1 on chip (else in HBM);
                                  2 if, besides, a single system on the sliced layout runs
                                  the two-barrier form (directions formed while gathered);
-                                 3 if it keeps r and q on chip and x, M^-1 in HBM (tiles
-                                 too large for three vectors on chip);
-                                 the environment variables SLA_GRID_ONCHIP=0, SLA_GRID2=0
-                                 and SLA_GRID_RQS=0, read at creation, turn these variants
-                                 off (SLA_GRID_ONCHIP=2 leaves only variant 3) */
+                                 the environment variables SLA_GRID_ONCHIP=0 and
+                                 SLA_GRID2=0, read at creation, turn these variants off */
     int32_t grid_tile_rows;   /* rows of one grid-solver tile (SLA_SELL_PACK=1, read at each
                                  solve, makes the sliced SpMV read value-and-column records,
                                  one load an entry; off by default, see the design notes) */
@@ -141,7 +138,9 @@ typedef struct {
                                  extra value-gather kernel per solve); 2 if, besides,
                                  every slice is padded to the widest row (padding at most
                                  3 % of the entries; SLA_SELL_UNIFORM=0, read at creation,
-                                 turns this off) */
+                                 turns this off); 3 if the rows of each 32-row window are
+                                 ordered by length before slicing (irregular rows, vectors
+                                 in HBM; SLA_SELL_SORT=0 turns this off) */
     int32_t block_resident;   /* 1 if the block solver keeps values and pattern of a
                                  system in shared memory as well as its vectors */
     int32_t cluster_fits;     /* 1 if one system fits the cluster solver */
@@ -149,6 +148,10 @@ typedef struct {
     int32_t item_rows_max;    /* list handles: rows of the largest item */
     int32_t item_smem_rows;   /* list handles: items up to this size keep their vectors in
                                  shared memory (larger ones use the workspace) */
+    int32_t sliced_col_bytes; /* bytes a column of the sliced layout takes in the solver's
+                                 matrix stream: 2 when every |column - row| < 2^15 (16-bit
+                                 offsets from the row; SLA_SELL_D16=0, read at creation,
+                                 turns them off), else 4; 0 without the sliced layout */
     int32_t interleaved;      /* 1 if forward (and symmetric adjoint) grid solves of this
                                  batch of 2 or 4 systems run the interleaved solver: values
                                  [entry][system] and vectors [row][system] in the workspace,

@@ -5,8 +5,9 @@ index a kernel takes from the pattern, and every shared-memory or cluster-rank
 index derived from one, is checked before use and recorded instead of used when
 out of range.  Runs every solver form on small systems (thread-block cluster,
 block per system with and without the matrix in shared memory, persistent grid
-with vectors on chip, r and q on chip or all in HBM, sliced (uniform or
-per-slice widths) or CSR rows, two-barrier form, the
+with vectors on chip (own p too, or not) or in HBM, sliced (uniform or
+per-slice widths, rows sorted within windows, 16- or 32-bit columns) or CSR
+rows, two-barrier form, the
 interleaved batch, lists of systems, the allocation-free entry point), the
 adjoints (symmetric and through A^T's pattern), SpMV both ways, both value
 gradients and the edge-weighted Laplacian; compares each result with the CPU
@@ -97,17 +98,16 @@ def main():
     w = W.c3_diffusion3d(N=40)
     for label, env in (("3-D grid on chip, two barriers", {}),
                        ("3-D grid on chip, three barriers", {"SLA_GRID2": "0"}),
-                       ("3-D grid, r and q on chip", {"SLA_GRID_ONCHIP": "2"}),
-                       ("3-D grid, r and q on chip, per-slice widths", {"SLA_GRID_ONCHIP": "2",
-                                                                       "SLA_SELL_UNIFORM": "0"}),
+                       ("3-D grid, HBM, per-slice widths", {"SLA_GRID_ONCHIP": "0", "SLA_SELL_UNIFORM": "0"}),
                        ("3-D grid, vectors in HBM, sliced", {"SLA_GRID_ONCHIP": "0"}),
                        ("3-D grid, vectors in HBM, CSR rows", {"SLA_GRID_ONCHIP": "0", "SLA_SELL": "0"}),
-                       ("3-D grid, HBM, L2 prefetch", {"SLA_GRID_ONCHIP": "0", "SLA_L2_PREFETCH": "2"})):
+                       ("3-D grid, HBM, 32-bit columns", {"SLA_GRID_ONCHIP": "0", "SLA_SELL_D16": "0"}),
+                       ("3-D grid on chip, own p in HBM", {"SLA_GRID2": "0", "SLA_GRID_P4": "0"})):
         pipeline(label, w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,
                  strategy=L.SLA_STRATEGY_GRID, env=env)
-    rp, ci, v = W.random_spd(3000, 0.002, 8, diag_extra=0.3)     # irregular rows: sorted windows
+    rp, ci, v = W.random_spd(12000, 0.0005, 9, diag_extra=0.3)   # irregular rows: sorted windows
     pipeline("irregular rows, vectors in HBM, sorted windows", rp, ci, v[None, :],
-             W.uniform(8, 0, 3000, -1, 1)[None, :], W.uniform(8, 1, 3000, -1, 1)[None, :], fixed_iters=30,
+             W.uniform(8, 0, 12000, -1, 1)[None, :], W.uniform(8, 1, 12000, -1, 1)[None, :], fixed_iters=30,
              strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0"})
     w = W.c3_batched(N=24, B=2)
     pipeline("interleaved batch of 2", w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,

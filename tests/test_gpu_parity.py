@@ -282,6 +282,9 @@ def _cases():
     yield "poisson37", rp, ci, v[None, :], W.normal(5, 0, 37 * 37)[None, :]
     rp, ci, v = W.random_spd(3000, 0.002, 8, diag_extra=0.3)   # varying diagonal
     yield "random3000", rp, ci, v[None, :], W.uniform(8, 0, 3000, -1, 1)[None, :]
+    # irregular rows in tiles of at least 32 rows: the sorted-window sliced layout
+    rp, ci, v = W.random_spd(12000, 0.0005, 9, diag_extra=0.3)
+    yield "random12000", rp, ci, v[None, :], W.uniform(9, 0, 12000, -1, 1)[None, :]
     rp, ci, v = _spd_long_rows(6000, 60, 3)              # wide rows: several lanes a row
     yield "wide6000", rp, ci, v[None, :], W.uniform(3, 0, 6000, -1, 1)[None, :]
     w = W.c4_batched(B=24)
@@ -289,25 +292,28 @@ def _cases():
 
 
 # (strategy, on-chip grid vectors, sliced short-row layout); on-chip "3" keeps
-# the vectors on chip but turns the two-barrier single-system form off; "2"
-# keeps only r and q on chip (x and M^-1 in HBM); sliced "u" is the sliced
+# the vectors on chip but turns the two-barrier single-system form off (the
+# tile's own p then also on chip where it fits), "4" as "3" without own p on chip; sliced "u" is the sliced
 # layout with per-slice widths (uniform widths off), "n" without the rows of
-# irregular patterns sorted by length within 32-row windows
+# irregular patterns sorted by length within 32-row windows, "w" with 32-bit
+# columns only (no 16-bit offsets)
 SOLVER_VARIANTS = [
-    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"),
+    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"), (L.SLA_STRATEGY_GRID, "4", "1"),
     (L.SLA_STRATEGY_GRID, "0", "1"), (L.SLA_STRATEGY_GRID, "1", "0"),
-    (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_GRID, "2", "1"),
-    (L.SLA_STRATEGY_GRID, "2", "0"), (L.SLA_STRATEGY_GRID, "1", "u"),
+    (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_GRID, "1", "u"),
     (L.SLA_STRATEGY_GRID, "0", "u"), (L.SLA_STRATEGY_GRID, "0", "n"),
+    (L.SLA_STRATEGY_GRID, "1", "w"), (L.SLA_STRATEGY_GRID, "0", "w"),
     (L.SLA_STRATEGY_BLOCK, "1", "1"), (L.SLA_STRATEGY_CLUSTER, "1", "1")]
 
 
 def _variant_env(monkeypatch, onchip, sell):
-    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip if onchip in ("0", "2") else "1")
-    monkeypatch.setenv("SLA_GRID2", "0" if onchip == "3" else "1")
+    monkeypatch.setenv("SLA_GRID_ONCHIP", "0" if onchip == "0" else "1")
+    monkeypatch.setenv("SLA_GRID2", "0" if onchip in ("3", "4") else "1")
+    monkeypatch.setenv("SLA_GRID_P4", "0" if onchip == "4" else "1")
     monkeypatch.setenv("SLA_SELL", "0" if sell == "0" else "1")
     monkeypatch.setenv("SLA_SELL_UNIFORM", "0" if sell == "u" else "1")
     monkeypatch.setenv("SLA_SELL_SORT", "0" if sell == "n" else "1")
+    monkeypatch.setenv("SLA_SELL_D16", "0" if sell == "w" else "1")
 
 
 @pytest.mark.parametrize("strategy,onchip,sell", SOLVER_VARIANTS)
@@ -327,17 +333,19 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
             continue
         if strategy == L.SLA_STRATEGY_GRID and onchip == "0":
             assert A.props.grid_onchip == 0
-        if strategy == L.SLA_STRATEGY_GRID and onchip == "3":
+        if strategy == L.SLA_STRATEGY_GRID and onchip in ("3", "4"):
             assert A.props.grid_onchip in (0, 1)
         if strategy == L.SLA_STRATEGY_GRID and onchip == "1" and B == 1 and A.props.sliced:
             assert A.props.grid_onchip == 2, name
-        if strategy == L.SLA_STRATEGY_GRID and onchip == "2":
-            assert A.props.grid_onchip == 3 or A.props.lanes > 1, name
         if sell == "u":
             assert A.props.sliced in (0, 1, 3), name
         if sell == "n":
             assert A.props.sliced in (0, 1, 2), name
-        if name == "random3000" and strategy == L.SLA_STRATEGY_GRID and onchip in ("0", "2") \
+        if sell == "w":
+            assert A.props.sliced_col_bytes in (0, 4), name
+        if name == "poisson37" and sell == "1":
+            assert A.props.sliced_col_bytes == 2, name       # offsets within +-37
+        if name == "random12000" and strategy == L.SLA_STRATEGY_GRID and onchip == "0" \
                 and sell in ("1", "u"):
             assert A.props.sliced == 3, name            # irregular rows: sorted windows
         for k in (1, 7, 60):
@@ -379,7 +387,7 @@ def test_grid_and_block_strategies_agree():
     assert np.all(np.abs(H(ig.iters) - H(ib.iters)) <= 2)
 
 
-@pytest.mark.parametrize("onchip", ["1", "0", "2"])
+@pytest.mark.parametrize("onchip", ["1", "0"])
 def test_results_are_bitwise_reproducible(onchip, monkeypatch):
     monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
     w = W.c1_poisson64()
@@ -484,7 +492,7 @@ def test_adjoint_memory_does_not_grow_with_iterations():
 
 # ------------------------------------------------------------ edge cases ----
 
-@pytest.mark.parametrize("onchip", ["1", "3", "2"])
+@pytest.mark.parametrize("onchip", ["1", "3", "0"])
 def test_edge_cases_match_oracle_outcomes(onchip, monkeypatch):
     _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.random_spd(300, 0.02, 4)
@@ -533,7 +541,7 @@ def test_single_unknown_and_empty_matrix():
     assert x.shape == (2, 0) and np.all(H(info.status) == 0) and np.all(H(info.iters) == 0)
 
 
-@pytest.mark.parametrize("onchip", ["1", "3", "0", "2"])
+@pytest.mark.parametrize("onchip", ["1", "3", "0"])
 def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
     _variant_env(monkeypatch, onchip, "1")
     rp, ci, v = W.poisson2d(300)
