@@ -77,7 +77,6 @@ struct CgArgs {
     int sell_w;         // > 0: every slice of the sliced layout is sell_w entries wide
     const int32_t *sell_perm;   // or null: the row at each position of the sliced layout
     const int16_t *sell_d16;    // or null: the sliced layout's columns as offsets from their row
-    int p_onchip;       // on-chip solver: the tile's own p also kept in shared memory
 };
 
 // ------------------------------------------------------------ helpers ----
@@ -326,10 +325,6 @@ cg_grid_kernel(CgArgs<T> a) {
     T *xs_ = reinterpret_cast<T *>(smem_raw);     // ONCHIP: [tile_rows] each
     T *rs_ = xs_ + (ONCHIP ? a.tile_rows : 0);
     T *ds_ = rs_ + (ONCHIP ? a.tile_rows : 0);
-    // ONCHIP with p_onchip: the tile's own rows of p, read by the p.q partials,
-    // x += alpha p and the direction update without a round trip to L2 (p is
-    // still written to global memory for the other tiles' gathers)
-    T *ps_ = (ONCHIP && a.p_onchip) ? ds_ + a.tile_rows : nullptr;
 
     if (blockIdx.x == 0 && tid == 0) a.sync[3] = (unsigned)a.B;
 
@@ -363,7 +358,6 @@ cg_grid_kernel(CgArgs<T> a) {
             const T zi = di * ri;
             pg[i] = zi;
             if constexpr (ONCHIP) {
-                if (ps_) ps_[i - r0] = zi;
                 xs_[i - r0] = xi;
                 rs_[i - r0] = ri;
                 ds_[i - r0] = di;
@@ -457,7 +451,7 @@ cg_grid_kernel(CgArgs<T> a) {
                         if (i < r1) {
                             const T qi = sell_row_rec<false>(a.sell_ptr, rec, pg, i, n, a.sell_nnz);
                             qreg[j] = qi;
-                            acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
+                            acc[0] += (double)pg[i] * (double)qi;
                         }
                     }
                 } else {
@@ -472,7 +466,7 @@ cg_grid_kernel(CgArgs<T> a) {
                                 : sell_row<0, false>(a.sell_ptr, a.sell_cols, a.sell_d16, svals, pg, i, i, n,
                                                      a.sell_nnz, a.sell_w);
                             qreg[j] = qi;
-                            acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
+                            acc[0] += (double)pg[i] * (double)qi;
                         }
                     }
                 }
@@ -483,7 +477,7 @@ cg_grid_kernel(CgArgs<T> a) {
                     if (i < r1) {
                         const T qi = row_dot<T, 1>(a.rowptr, a.colind, vs, pg, i, 0, n, a.nnz);
                         qreg[j] = qi;
-                        acc[0] += (double)(ps_ ? ps_[i - r0] : pg[i]) * (double)qi;
+                        acc[0] += (double)pg[i] * (double)qi;
                     }
                 }
             } else if constexpr (SELL) {
@@ -583,7 +577,7 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                 for (int j = 0; j < RPT; ++j) {
                     const int i = r0 + tid + j * NT;
-                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * (ps_ ? ps_[i - r0] : pg[i]);
+                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * pg[i];
                 }
             } else {
                 T *xg = a.x + (int64_t)s * n;
@@ -618,11 +612,7 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
-                        if (i < r1) {
-                            const T pn = ds_[i - r0] * rs_[i - r0] + bt * (ps_ ? ps_[i - r0] : pg[i]);
-                            pg[i] = pn;
-                            if (ps_) ps_[i - r0] = pn;
-                        }
+                        if (i < r1) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pg[i];
                     }
                 } else {
                     const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;
@@ -1844,7 +1834,7 @@ sla_status cg_configure(Csr *h) {
             for (int sv = 0; sv < 3; ++sv)
                 SLA_CHECK_CUDA(cudaFuncSetAttribute(
                     sv < 2 ? pick_onchip(h->dtype, rpt, sv != 0) : pick_grid2(h->dtype, rpt),
-                    cudaFuncAttributeMaxDynamicSharedMemorySize, sv < 2 ? optin - 4096 : optin - 16384));
+                    cudaFuncAttributeMaxDynamicSharedMemorySize, optin - 16384));
             const void *f = pick_onchip(h->dtype, rpt, true);
             int per_sm = 0;
             SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kOnchipThreads, smem));
@@ -1870,19 +1860,7 @@ sla_status cg_configure(Csr *h) {
                 const bool l1_fits = smem + 2 * (size_t)tr * ts <= (size_t)smem_sm;
                 h->grid2 = h->batch == 1 && nt <= h->num_sms && per_sm2 >= 1 &&
                            (l1_fits || (g2 && g2[0] == '2')) && !(g2 && g2[0] == '0');
-                // The three-barrier solver also keeps the tile's own p on chip when a
-                // fourth vector fits (SLA_GRID_P4=0 turns it off).
-                const char *p4 = getenv("SLA_GRID_P4");
-                h->p_onchip = false;
-                if (!h->grid2 && 4 * (size_t)tr * ts + 4096 <= (size_t)optin && !(p4 && p4[0] == '0')) {
-                    int per_sm4 = 0;
-                    SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                        &per_sm4, f, kOnchipThreads, 4 * (size_t)tr * ts));
-                    if (per_sm4 >= 1) {
-                        h->p_onchip = true;
-                        h->grid_smem = 4 * (size_t)tr * ts;
-                    }
-                }
+
             }
         }
     }
@@ -2101,7 +2079,6 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
     a.timeout_ns = o->wait_timeout_ns > 0 ? o->wait_timeout_ns : kDefaultTimeoutNs;
     a.tile_rows = h->tile_rows;
     a.ntiles = h->ntiles;
-    a.p_onchip = h->p_onchip ? 1 : 0;
     if (h->dep_lo != nullptr && pattern_is_forward_or_sym(h, rowptr)) {
         a.dep_lo = h->dep_lo;
         a.dep_hi = h->dep_hi;

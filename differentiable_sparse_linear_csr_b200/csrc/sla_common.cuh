@@ -108,7 +108,6 @@ struct Csr {
     bool onchip = false;               // grid solver keeps x, r, M^-1 in shared memory
     int32_t onchip_rpt = 0;            // rows a thread in the on-chip grid solver
     bool grid2 = false;                // single system, on chip, sliced: two barriers an iteration
-    bool p_onchip = false;             // on-chip solver keeps the tile's own p in shared memory too
     int32_t grid_threads = 0;          // threads of a grid-solver block
     size_t grid_smem = 0;              // dynamic shared memory of a grid-solver block
     size_t block_smem = 0;             // its dynamic shared memory per block

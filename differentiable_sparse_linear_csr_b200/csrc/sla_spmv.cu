@@ -4,27 +4,59 @@
 //   torch-sla summary page, technical summary: "Methodology" 1 (`.matvec`)
 //   and "Methodology" 2 (linear systems: gradient on the sparsity pattern).
 //
-// Short rows (one thread a row): a block takes 256 consecutive rows, whose
-// entries are one contiguous range of the CSR arrays.  The block copies that
-// range's column indices (and, per system, values) into shared memory with
-// coalesced loads, so every global read of the pattern and the values and
-// every gradient store is a whole-sector access; the per-row work then reads
-// shared memory and gathers x.  A row keeps its stored-order sum (the same
-// rounding as a thread walking the row in global memory).  Chunks whose range
-// exceeds the shared-memory capacity fall back to that direct walk.
-// Long rows (LANES > 1 threads a row) are walked by sub-warps, which already
-// read consecutive entries.
+// Short rows (one thread a row):
+//  - SpMV: a block takes 256 consecutive rows, whose entries are one contiguous
+//    range of the CSR arrays; it copies the range's columns and values into
+//    shared memory with coalesced loads, then each thread sums its own row
+//    there in stored order while gathering x (the rounding of a thread walking
+//    the row in global memory).  Gathering row by row keeps a warp's gathers of
+//    x together for banded patterns (consecutive rows reach consecutive
+//    columns); gathering entry by entry measured slower.
+//  - Value gradients: each warp takes 32 rows and walks their entry range in
+//    order, the row of each entry taken from a per-warp table, so column reads
+//    and gradient stores are coalesced.
+// Both issue a group of kStage loads into registers before using any, so that
+// they are in flight together.  A block or warp whose range exceeds its shared
+// memory walks its rows in global memory.  Long rows (LANES > 1 threads a row)
+// are walked by sub-warps, which already read consecutive entries.
 #include "sla_rows.cuh"
 
 namespace sla {
 
-constexpr int kChunkRows = 256;          // rows (and threads) of one staged block
+constexpr int kChunkRows = 256;          // rows (and threads) of one staged SpMV block
+constexpr int kWarpRows = 32;            // rows of one warp in the one-thread-row gradient
+constexpr int kRowWarps = 8;             // warps of one block there
+constexpr int kStage = 4;                // loads issued before any is used
 
-// Entries a staged block holds: room for rows 4 entries longer than the mean,
-// at most 4096; a chunk with more entries walks its rows in global memory.
+// Entries a staged SpMV block holds: room for rows 4 entries longer than the
+// mean, at most 4096; a chunk with more walks its rows in global memory.
 static int chunk_cap(double row_mean) {
     const double c = kChunkRows * (row_mean + 4.0);
     return c >= 4096.0 ? 4096 : ((int)c + 31) / 32 * 32;
+}
+
+static dim3 chunk_grid(int rows, int B) {
+    return dim3((unsigned)((rows + kChunkRows - 1) / kChunkRows), (unsigned)(B < 65535 ? B : 65535));
+}
+
+// Entries one gradient warp tabulates: room for rows 4 entries longer than
+// the mean, at most 1024; a warp with more walks its rows in global memory.
+// A product rounded on its own (the compiler must not fuse it into a
+// following add), as the gradient's definition rounds it.
+template <typename T>
+__device__ __forceinline__ T mul_rn(T a, T b) {
+    if constexpr (sizeof(T) == 8) return __dmul_rn(a, b);
+    else return __fmul_rn(a, b);
+}
+
+static int warp_cap(double row_mean) {
+    const double c = kWarpRows * (row_mean + 4.0);
+    return c >= 1024.0 ? 1024 : ((int)c + 31) / 32 * 32;
+}
+
+static dim3 warp_grid(int rows, int B) {
+    const int rpb = kWarpRows * kRowWarps;
+    return dim3((unsigned)((rows + rpb - 1) / rpb), (unsigned)(B < 65535 ? B : 65535));
 }
 
 template <typename T, int LANES, bool PERM>
@@ -50,8 +82,8 @@ spmv_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32_t *__r
     }
 }
 
-// y = alpha A x + beta y for one-thread rows, the chunk's pattern and values
-// staged in shared memory (see the file comment).
+// y = alpha A x + beta y for one-thread rows, 256 rows a block (see the file
+// comment).
 template <typename T>
 __global__ void __launch_bounds__(kChunkRows)
 spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32_t *__restrict__ rowptr,
@@ -66,22 +98,48 @@ spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32
     const int e0 = __ldg(rowptr + r0), e1 = __ldg(rowptr + r1);
     const int t0 = i < r1 ? __ldg(rowptr + i) : 0, t1 = i < r1 ? __ldg(rowptr + i + 1) : 0;
     const bool staged = e1 - e0 <= cap;
-    if (staged) {
-#pragma unroll 4
-        for (int t = e0 + tid; t < e1; t += kChunkRows)
-            s_cols[t - e0] = __ldg(colind + SLA_IDX(t, nnz, kBndEntry));
-    }
     for (int sys = blockIdx.y; sys < B; sys += gridDim.y) {
         const T *vb = vals + (int64_t)sys * nnz;
         const T *xb = x + (int64_t)sys * x_stride;
         T s = T(0);
         if (staged) {
-#pragma unroll 4
-            for (int t = e0 + tid; t < e1; t += kChunkRows) s_vals[t - e0] = __ldg(vb + SLA_IDX(t, nnz, kBndEntry));
+            for (int base = e0 + tid; base < e1; base += kChunkRows * kStage) {
+                int c[kStage];
+                T v[kStage];
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) {
+                    const int t = base + kChunkRows * u;
+                    if (t < e1) {
+                        const int tt = SLA_IDX(t, nnz, kBndEntry);
+                        c[u] = __ldg(colind + tt);
+                        v[u] = __ldg(vb + tt);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) {
+                    const int t = base + kChunkRows * u;
+                    if (t < e1) {
+                        s_cols[t - e0] = c[u];
+                        s_vals[t - e0] = v[u];
+                    }
+                }
+            }
             __syncthreads();
-#pragma unroll 4
-            for (int t = t0; t < t1; ++t)
-                s += s_vals[t - e0] * __ldg(xb + SLA_IDX(s_cols[t - e0], x_stride, kBndColumn));
+            for (int t = t0; t < t1; t += kStage) {
+                T v[kStage], xv[kStage];
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) {
+                    v[u] = T(0);
+                    xv[u] = T(0);
+                    if (t + u < t1) {
+                        v[u] = s_vals[t + u - e0];
+                        xv[u] = __ldg(xb + SLA_IDX(s_cols[t + u - e0], x_stride, kBndColumn));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kStage; ++u)
+                    if (t + u < t1) s += v[u] * xv[u];
+            }
             __syncthreads();
         } else {
             for (int t = t0; t < t1; ++t) {
@@ -114,50 +172,75 @@ grad_values_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__
         T *gb = grad + (int64_t)sys * nnz;
         for (int t = t0 + lane; t < t1; t += LANES) {
             const int tt = SLA_IDX(t, nnz, kBndEntry);
-            const T p = li * __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn));
+            const T p = mul_rn(li, __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn)));
             const T g = NEG ? -p : p;
             gb[tt] = accumulate ? gb[tt] + g : g;
         }
     }
 }
 
-// The same for one-thread rows, entry-parallel over the chunk: each thread
-// first marks the chunk slots of its row with the row's position, then the
-// block walks the slots in order, so column reads and gradient stores are
-// coalesced.  Each entry is the same single product as above.
+// The same for one-thread rows, a warp per 32 rows: each lane marks the
+// warp's table slots of its row with its lane, then the warp walks the entry
+// range in order, so column reads and gradient stores are coalesced (loads of
+// a group of kStage steps in registers before any is used).  Each entry is the
+// same single product as above.
 template <typename T, bool NEG>
-__global__ void __launch_bounds__(kChunkRows)
-grad_staged_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__restrict__ rowptr,
-                   const int32_t *__restrict__ colind, const T *__restrict__ lam,
-                   const T *__restrict__ x, T *__restrict__ grad, int accumulate, int cap) {
-    extern __shared__ uint8_t s_row[];   // [cap]: position of each slot's row in the chunk
-    const int tid = threadIdx.x;
-    const int r0 = blockIdx.x * kChunkRows, r1 = min(n_rows, r0 + kChunkRows);
-    const int i = r0 + tid;
-    const int e0 = __ldg(rowptr + r0), e1 = __ldg(rowptr + r1);
+__global__ void __launch_bounds__(kWarpRows * kRowWarps)
+grad_warp_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__restrict__ rowptr,
+                 const int32_t *__restrict__ colind, const T *__restrict__ lam,
+                 const T *__restrict__ x, T *__restrict__ grad, int accumulate, int cap) {
+    extern __shared__ uint8_t s_all[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t *s_row = s_all + (size_t)warp * cap;   // [cap]: lane (row) of each entry
+    const int r0 = (blockIdx.x * kRowWarps + warp) * kWarpRows;
+    if (r0 >= n_rows) return;
+    const int r1 = min(n_rows, r0 + kWarpRows);
+    const int i = r0 + lane;
     const int t0 = i < r1 ? __ldg(rowptr + i) : 0, t1 = i < r1 ? __ldg(rowptr + i + 1) : 0;
+    const int e0 = __ldg(rowptr + r0), e1 = __ldg(rowptr + r1);
     const bool staged = e1 - e0 <= cap;
     if (staged) {
-        for (int t = t0; t < t1; ++t) s_row[t - e0] = (uint8_t)tid;
-        __syncthreads();
+        for (int t = t0; t < t1; ++t) s_row[t - e0] = (uint8_t)lane;
+        __syncwarp();
     }
     for (int sys = blockIdx.y; sys < B; sys += gridDim.y) {
         const T *lb = lam + (int64_t)sys * n_rows + r0;
         const T *xb = x + (int64_t)sys * n_cols;
         T *gb = grad + (int64_t)sys * nnz;
         if (staged) {
-#pragma unroll 4
-            for (int t = e0 + tid; t < e1; t += kChunkRows) {
-                const int tt = SLA_IDX(t, nnz, kBndEntry);
-                const T p = __ldg(lb + s_row[t - e0]) * __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn));
-                const T g = NEG ? -p : p;
-                gb[tt] = accumulate ? gb[tt] + g : g;
+            for (int base = e0 + lane; base < e1; base += 32 * kStage) {
+                int c[kStage];
+                T li[kStage], xv[kStage], old[kStage];
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) {
+                    const int t = base + 32 * u;
+                    c[u] = 0;
+                    li[u] = T(0);
+                    old[u] = T(0);
+                    if (t < e1) {
+                        const int tt = SLA_IDX(t, nnz, kBndEntry);
+                        c[u] = SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn);
+                        li[u] = __ldg(lb + s_row[t - e0]);
+                        if (accumulate) old[u] = gb[tt];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) xv[u] = base + 32 * u < e1 ? __ldg(xb + c[u]) : T(0);
+#pragma unroll
+                for (int u = 0; u < kStage; ++u) {
+                    const int t = base + 32 * u;
+                    if (t < e1) {
+                        const T p = mul_rn(li[u], xv[u]);   // rounded on its own, never fused
+                        const T g = NEG ? -p : p;
+                        gb[t] = accumulate ? old[u] + g : g;
+                    }
+                }
             }
         } else if (i < r1) {
-            const T li = __ldg(lb + tid);
+            const T l = __ldg(lb + lane);
             for (int t = t0; t < t1; ++t) {
                 const int tt = SLA_IDX(t, nnz, kBndEntry);
-                const T p = li * __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn));
+                const T p = mul_rn(l, __ldg(xb + SLA_IDX(__ldg(colind + tt), n_cols, kBndColumn)));
                 const T g = NEG ? -p : p;
                 gb[tt] = accumulate ? gb[tt] + g : g;
             }
@@ -170,10 +253,6 @@ static dim3 row_grid(int rows, int lanes, int B) {
     return dim3((unsigned)((rows + rpb - 1) / rpb), (unsigned)(B < 65535 ? B : 65535));
 }
 
-static dim3 chunk_grid(int rows, int B) {
-    return dim3((unsigned)((rows + kChunkRows - 1) / kChunkRows), (unsigned)(B < 65535 ? B : 65535));
-}
-
 template <bool NEG>
 static sla_status grad_entry(const char *name, sla_csr_t hh, const void *u, const void *x, void *grad,
                              int32_t accumulate, void *stream) {
@@ -184,14 +263,15 @@ static sla_status grad_entry(const char *name, sla_csr_t hh, const void *u, cons
     SLA_REQUIRE(u && x && grad, "%s: NULL vector or grad", name);
     cudaStream_t s = as_stream(stream);
     if (h->lanes == 1) {
-        const dim3 grid = chunk_grid(h->n_rows, h->batch);
-        const int cap = chunk_cap(h->row_mean);
+        const dim3 grid = warp_grid(h->n_rows, h->batch);
+        const int cap = warp_cap(h->row_mean);
+        const size_t smem = (size_t)cap * kRowWarps;
         if (h->dtype == SLA_F64)
-            grad_staged_kernel<double, NEG><<<grid, kChunkRows, cap, s>>>(
+            grad_warp_kernel<double, NEG><<<grid, kWarpRows * kRowWarps, smem, s>>>(
                 h->n_rows, h->n_cols, h->nnz, h->batch, h->rowptr, h->colind, (const double *)u,
                 (const double *)x, (double *)grad, accumulate, cap);
         else
-            grad_staged_kernel<float, NEG><<<grid, kChunkRows, cap, s>>>(
+            grad_warp_kernel<float, NEG><<<grid, kWarpRows * kRowWarps, smem, s>>>(
                 h->n_rows, h->n_cols, h->nnz, h->batch, h->rowptr, h->colind, (const float *)u,
                 (const float *)x, (float *)grad, accumulate, cap);
         SLA_CHECK_LAUNCH();

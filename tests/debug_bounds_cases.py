@@ -5,7 +5,7 @@ index a kernel takes from the pattern, and every shared-memory or cluster-rank
 index derived from one, is checked before use and recorded instead of used when
 out of range.  Runs every solver form on small systems (thread-block cluster,
 block per system with and without the matrix in shared memory, persistent grid
-with vectors on chip (own p too, or not) or in HBM, sliced (uniform or
+with vectors on chip or in HBM, tile flags or a third barrier, sliced (uniform or
 per-slice widths, rows sorted within windows, 16- or 32-bit columns) or CSR
 rows, two-barrier form, the
 interleaved batch, lists of systems, the allocation-free entry point), the
@@ -102,7 +102,8 @@ def main():
                        ("3-D grid, vectors in HBM, sliced", {"SLA_GRID_ONCHIP": "0"}),
                        ("3-D grid, vectors in HBM, CSR rows", {"SLA_GRID_ONCHIP": "0", "SLA_SELL": "0"}),
                        ("3-D grid, HBM, 32-bit columns", {"SLA_GRID_ONCHIP": "0", "SLA_SELL_D16": "0"}),
-                       ("3-D grid on chip, own p in HBM", {"SLA_GRID2": "0", "SLA_GRID_P4": "0"})):
+                       ("3-D grid on chip, three barriers, no tile flags", {"SLA_GRID2": "0",
+                                                                           "SLA_TILE_FLAGS": "0"})):
         pipeline(label, w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,
                  strategy=L.SLA_STRATEGY_GRID, env=env)
     rp, ci, v = W.random_spd(12000, 0.0005, 9, diag_extra=0.3)   # irregular rows: sorted windows

@@ -292,13 +292,12 @@ def _cases():
 
 
 # (strategy, on-chip grid vectors, sliced short-row layout); on-chip "3" keeps
-# the vectors on chip but turns the two-barrier single-system form off (the
-# tile's own p then also on chip where it fits), "4" as "3" without own p on chip; sliced "u" is the sliced
+# the vectors on chip but turns the two-barrier single-system form off; sliced "u" is the sliced
 # layout with per-slice widths (uniform widths off), "n" without the rows of
 # irregular patterns sorted by length within 32-row windows, "w" with 32-bit
 # columns only (no 16-bit offsets)
 SOLVER_VARIANTS = [
-    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"), (L.SLA_STRATEGY_GRID, "4", "1"),
+    (L.SLA_STRATEGY_GRID, "1", "1"), (L.SLA_STRATEGY_GRID, "3", "1"),
     (L.SLA_STRATEGY_GRID, "0", "1"), (L.SLA_STRATEGY_GRID, "1", "0"),
     (L.SLA_STRATEGY_GRID, "0", "0"), (L.SLA_STRATEGY_GRID, "1", "u"),
     (L.SLA_STRATEGY_GRID, "0", "u"), (L.SLA_STRATEGY_GRID, "0", "n"),
@@ -308,8 +307,7 @@ SOLVER_VARIANTS = [
 
 def _variant_env(monkeypatch, onchip, sell):
     monkeypatch.setenv("SLA_GRID_ONCHIP", "0" if onchip == "0" else "1")
-    monkeypatch.setenv("SLA_GRID2", "0" if onchip in ("3", "4") else "1")
-    monkeypatch.setenv("SLA_GRID_P4", "0" if onchip == "4" else "1")
+    monkeypatch.setenv("SLA_GRID2", "0" if onchip == "3" else "1")
     monkeypatch.setenv("SLA_SELL", "0" if sell == "0" else "1")
     monkeypatch.setenv("SLA_SELL_UNIFORM", "0" if sell == "u" else "1")
     monkeypatch.setenv("SLA_SELL_SORT", "0" if sell == "n" else "1")
@@ -333,7 +331,7 @@ def test_pcg_fixed_iterations_parity(strategy, onchip, sell, dtype, monkeypatch)
             continue
         if strategy == L.SLA_STRATEGY_GRID and onchip == "0":
             assert A.props.grid_onchip == 0
-        if strategy == L.SLA_STRATEGY_GRID and onchip in ("3", "4"):
+        if strategy == L.SLA_STRATEGY_GRID and onchip == "3":
             assert A.props.grid_onchip in (0, 1)
         if strategy == L.SLA_STRATEGY_GRID and onchip == "1" and B == 1 and A.props.sliced:
             assert A.props.grid_onchip == 2, name
@@ -544,14 +542,15 @@ def test_single_unknown_and_empty_matrix():
 @pytest.mark.parametrize("onchip", ["1", "3", "0"])
 def test_bounded_wait_times_out_without_hanging(onchip, monkeypatch):
     _variant_env(monkeypatch, onchip, "1")
-    rp, ci, v = W.poisson2d(300)
+    N = 1024                          # one tile a block: tile flags in place of a barrier
+    rp, ci, v = W.poisson2d(N)
     A = make(rp, ci)
-    b = T(W.normal(2, 0, 300 * 300))
+    b = T(W.normal(2, 0, N * N))
     _, info = A.cg(T(v), b, fixed_iters=500, strategy=L.SLA_STRATEGY_GRID, wait_timeout_ns=1)
     assert H(info.status)[0] == L.SLA_TIMED_OUT
     # the context is still usable and a normal solve is correct afterwards
     x, info = A.cg(T(v), b, fixed_iters=20, strategy=L.SLA_STRATEGY_GRID)
-    xo, _ = O.pcg(rp, ci, v, W.normal(2, 0, 300 * 300), fixed_iters=20)
+    xo, _ = O.pcg(rp, ci, v, W.normal(2, 0, N * N), fixed_iters=20)
     assert H(info.status)[0] == L.SLA_FIXED_DONE and rel(H(x)[0], xo) < TOL_X64
 
 
