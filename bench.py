@@ -368,8 +368,19 @@ def spmv_block(A, vals, n: int, nnz: int, B: int, vbytes: int, dt, dev, flush, p
     ms = time_kernel_ms(lambda: L.sla_spmv(A.handle, vals, x, y, 0, 1.0, 0.0), flush)
     by = spmv_bytes(n, nnz, vbytes) * B
     gbs = by / (ms / 1000.0) / 1e9
+    # context for a launch this short: torch's own reduction reading the same
+    # number of bytes, timed the same way (the same L2 flush before each)
+    buf = torch.empty(by // 8, dtype=torch.float64, device=dev).uniform_()
+    ms_read = time_kernel_ms(lambda: torch.sum(buf), flush)
+    read_gbs = by / (ms_read / 1000.0) / 1e9
+    del buf
+    kernel = ("sla_spmv, pipelined one-thread rows: 256-row chunks copied to shared memory one chunk "
+              "ahead (cp.async)" if vbytes == 8 else
+              "sla_spmv, one-thread rows: 256-row chunks staged in shared memory")
     return {"ms": ms, "algorithmic_bytes": by, "gbs": gbs, "frac_of_hbm_peak": gbs / peak,
-            "kernel": "sla_spmv (one-thread rows: 256-row chunks staged in shared memory)"}
+            "same_bytes_read_gbs": read_gbs, "frac_of_same_bytes_read": gbs / read_gbs,
+            "same_bytes_read": "torch.sum over a buffer of the same bytes, same flush before each",
+            "kernel": kernel}
 
 
 def l2_stream_peak_gbs(dev) -> float:

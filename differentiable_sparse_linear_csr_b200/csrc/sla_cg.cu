@@ -322,6 +322,11 @@ cg_grid_kernel(CgArgs<T> a) {
     const int n = a.n;
     unsigned target = 0;
     T qreg[ONCHIP ? RPT : 1];
+    // ONCHIP fp32: the tile's p, read once for x += alpha p and kept in
+    // registers for the direction update (q's registers are free again by
+    // then); fp64 keeps re-reading it (two more registers a row spill there)
+    constexpr bool KEEP_P = ONCHIP && sizeof(T) == 4;
+    T preg[KEEP_P ? RPT : 1];
     T *xs_ = reinterpret_cast<T *>(smem_raw);     // ONCHIP: [tile_rows] each
     T *rs_ = xs_ + (ONCHIP ? a.tile_rows : 0);
     T *ds_ = rs_ + (ONCHIP ? a.tile_rows : 0);
@@ -577,7 +582,11 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                 for (int j = 0; j < RPT; ++j) {
                     const int i = r0 + tid + j * NT;
-                    if (i < r1) xs_[i - r0] = xs_[i - r0] + al * pg[i];
+                    if (i < r1) {
+                        const T pj = pg[i];
+                        if constexpr (KEEP_P) preg[j] = pj;
+                        xs_[i - r0] = xs_[i - r0] + al * pj;
+                    }
                 }
             } else {
                 T *xg = a.x + (int64_t)s * n;
@@ -612,7 +621,12 @@ cg_grid_kernel(CgArgs<T> a) {
 #pragma unroll
                     for (int j = 0; j < RPT; ++j) {
                         const int i = r0 + tid + j * NT;
-                        if (i < r1) pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pg[i];
+                        if (i < r1) {
+                            T pj;
+                            if constexpr (KEEP_P) pj = preg[j];
+                            else pj = pg[i];
+                            pg[i] = ds_[i - r0] * rs_[i - r0] + bt * pj;
+                        }
                     }
                 } else {
                     const T *rg = a.r + (int64_t)s * n, *dg = a.d + (int64_t)s * n;

@@ -140,6 +140,9 @@ struct Csr {
     int32_t *sell_ptr = nullptr;       // owned [n_slices + 1]: first entry of each slice
     int32_t *sell_cols = nullptr;      // owned [sell_nnz]: column (own row for padding)
     int32_t *sell_map = nullptr;       // owned [sell_nnz]: CSR position, -1 for padding
+    // Grid of the pipelined one-thread-row SpMV (blocks resident at once; 0
+    // until first used).
+    int32_t pipe_grid_spmv = 0;
 };
 
 inline size_t dtype_size(sla_dtype dt) { return dt == SLA_F64 ? 8 : 4; }

@@ -12,6 +12,7 @@
 //    the row in global memory).  Gathering row by row keeps a warp's gathers of
 //    x together for banded patterns (consecutive rows reach consecutive
 //    columns); gathering entry by entry measured slower.
+//    fp64 values take a pipelined form of this (after the staged kernel).
 //  - Value gradients: each warp takes 32 rows and walks their entry range in
 //    order, the row of each entry taken from a per-warp table, so column reads
 //    and gradient stores are coalesced.
@@ -26,12 +27,14 @@ namespace sla {
 constexpr int kChunkRows = 256;          // rows (and threads) of one staged SpMV block
 constexpr int kWarpRows = 32;            // rows of one warp in the one-thread-row gradient
 constexpr int kRowWarps = 8;             // warps of one block there
-constexpr int kStage = 4;                // loads issued before any is used
+constexpr int kStage = 8;                // SpMV: loads issued before any is used
+constexpr int kGradStage = 4;            // the same for the gradient (more registers a step)
 
-// Entries a staged SpMV block holds: room for rows 4 entries longer than the
-// mean, at most 4096; a chunk with more walks its rows in global memory.
+// Entries a staged SpMV block holds: room for rows 2 entries longer than the
+// mean (so that 8 blocks fit an SM for rows of 7), at most 4096; a chunk with
+// more walks its rows in global memory.
 static int chunk_cap(double row_mean) {
-    const double c = kChunkRows * (row_mean + 4.0);
+    const double c = kChunkRows * (row_mean + 2.0);
     return c >= 4096.0 ? 4096 : ((int)c + 31) / 32 * 32;
 }
 
@@ -154,6 +157,167 @@ spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32
     }
 }
 
+// ---- pipelined one-thread-row SpMV (fp64) --------------------------------
+// A block stays resident and takes the chunks (kChunkRows consecutive rows of
+// one system) blockIdx.x, blockIdx.x + gridDim.x, ... .  A chunk's entries are
+// one contiguous range of the CSR arrays: its values, columns and row pointers
+// are copied into one of kPipe shared-memory stages by 16-byte asynchronous
+// copies (cp.async, cached in L2 only), issued one chunk ahead of the chunk
+// being summed, so the block's next HBM reads are in flight while it gathers x
+// for the current chunk.  Each copied range starts at its first byte rounded
+// down to 16 (the arrays start on 16-byte boundaries) and reads nothing past
+// the array's end.  A chunk with more entries than a stage holds walks its
+// rows in global memory (its row pointers are still staged).  Two stages keep
+// three blocks (24 warps) on an SM for rows of 7; three stages (two chunks
+// ahead) left room for two blocks and measured slower, and so did the same
+// pipeline for the value gradient and for fp32 SpMV on the 2-D Poisson matrix.
+
+constexpr int kPipe = 2;                 // stages: the chunk in flight + the one being summed
+
+__host__ __device__ constexpr int pipe_region(int64_t bytes) {
+    return (int)((bytes + 32 + 15) / 16 * 16);   // the range plus both roundings
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Queue the copy of bytes [lo, hi) of an array ending at `end` to shared
+// address dst (from lo rounded down to 16); 16 bytes a thread-step, the last
+// piece cut at `end` (cp.async fills the rest of it with zeros).
+__device__ __forceinline__ void stage_range(uint32_t dst, const void *lo, const void *hi, const void *end,
+                                            int tid) {
+    const uintptr_t a0 = (uintptr_t)lo & ~(uintptr_t)15;
+    const int pieces = (int)(((uintptr_t)hi - a0 + 15) >> 4);
+    for (int q = tid; q < pieces; q += kChunkRows) {
+        const uintptr_t src = a0 + 16 * (uintptr_t)q;
+        const uintptr_t left = (uintptr_t)end - src;
+        cp_async16(dst + 16 * q, (const void *)src, left >= 16 ? 16 : (int)left);
+    }
+}
+
+// Element offset of p within its 16-byte line.
+template <typename E>
+__device__ __forceinline__ int line_off(const E *p) {
+    return (int)(((uintptr_t)p & 15) / sizeof(E));
+}
+
+// Byte sizes of one stage's regions: values (VB bytes an entry), columns, row
+// pointers.
+struct PipeStage {
+    int rv, rc, rr;
+    __host__ __device__ PipeStage(int cap, int vb)
+        : rv(pipe_region((int64_t)cap * vb)), rc(pipe_region((int64_t)cap * 4)),
+          rr(pipe_region((int64_t)(kChunkRows + 1) * 4)) {}
+    __host__ __device__ int bytes() const { return rv + rc + rr; }
+};
+
+// Queue a chunk's copies (rows from r0, entries [e0, e1), values of its system
+// from vb) into the stage at shared address st.
+template <typename T>
+__device__ __forceinline__ void pipe_issue(uint32_t st, const PipeStage &L, int cap, int n_rows,
+                                           int64_t nnz, int r0, int e0, int e1,
+                                           const int32_t *__restrict__ rowptr,
+                                           const int32_t *__restrict__ colind, const T *vb, int tid) {
+    const int r1 = min(n_rows, r0 + kChunkRows);
+    stage_range(st + L.rv + L.rc, rowptr + r0, rowptr + r1 + 1, rowptr + n_rows + 1, tid);
+    if (e1 - e0 <= cap) {
+        stage_range(st, vb + e0, vb + e1, vb + nnz, tid);
+        stage_range(st + L.rv, colind + e0, colind + e1, colind + nnz, tid);
+    }
+}
+
+// y = alpha A x + beta y (one-thread rows), pipelined as above.  Each thread
+// sums its row in stored order, like every other one-thread-row kernel.
+template <typename T>
+__global__ void __launch_bounds__(kChunkRows)
+spmv_pipe_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32_t *__restrict__ rowptr,
+                 const int32_t *__restrict__ colind, const T *__restrict__ vals,
+                 const T *__restrict__ x, T *__restrict__ y, T alpha, T beta, int cap) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int tid = threadIdx.x;
+    const PipeStage L(cap, (int)sizeof(T));
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem_raw);
+    const int nchunks = (n_rows + kChunkRows - 1) / kChunkRows;
+    const int64_t units = (int64_t)nchunks * B;
+    const int64_t G = gridDim.x;
+    const int mine = blockIdx.x < units ? (int)((units - blockIdx.x + G - 1) / G) : 0;
+    // entry range of my k-th chunk (read one iteration before its copy is queued)
+    auto range = [&](int k, int &e0, int &e1) {
+        if (k >= mine) return;
+        const int r0 = (int)((blockIdx.x + k * G) % nchunks) * kChunkRows;
+        e0 = SLA_IDX(__ldg(rowptr + r0), nnz + 1, kBndEntry);
+        e1 = SLA_IDX(__ldg(rowptr + min(n_rows, r0 + kChunkRows)), nnz + 1, kBndEntry);
+    };
+    auto issue = [&](int k, int e0, int e1) {
+        if (k >= mine) return;
+        const int64_t u = blockIdx.x + k * G;
+        const int sys = (int)(u / nchunks), r0 = (int)(u % nchunks) * kChunkRows;
+        pipe_issue<T>(sbase + (k % kPipe) * L.bytes(), L, cap, n_rows, nnz, r0, e0, e1, rowptr, colind,
+                      vals + (int64_t)sys * nnz, tid);
+    };
+    int ne0 = 0, ne1 = 0;
+#pragma unroll
+    for (int k = 0; k < kPipe - 1; ++k) {
+        range(k, ne0, ne1);
+        issue(k, ne0, ne1);
+        cp_async_commit();
+    }
+    range(kPipe - 1, ne0, ne1);
+    for (int j = 0; j < mine; ++j) {
+        cp_async_wait<kPipe - 2>();   // chunk j's copies (this thread's) have landed
+        __syncthreads();              // everyone's have; chunk j - 1's stage is free
+        issue(j + kPipe - 1, ne0, ne1);
+        cp_async_commit();
+        range(j + kPipe, ne0, ne1);
+        const int64_t u = blockIdx.x + j * G;
+        const int sys = (int)(u / nchunks), r0 = (int)(u % nchunks) * kChunkRows;
+        const int r1 = min(n_rows, r0 + kChunkRows), i = r0 + tid;
+        unsigned char *stage = smem_raw + (j % kPipe) * L.bytes();
+        const int32_t *srp = reinterpret_cast<const int32_t *>(stage + L.rv + L.rc) + line_off(rowptr + r0);
+        const int e0 = srp[0], e1 = srp[r1 - r0];
+        const T *vb = vals + (int64_t)sys * nnz;
+        const T *xb = x + (int64_t)sys * x_stride;
+        if (i >= r1) continue;
+        const int t0 = srp[tid], t1 = srp[tid + 1];
+        T s = T(0);
+        if (e1 - e0 <= cap) {
+            const T *sv = reinterpret_cast<const T *>(stage) + line_off(vb + e0) - e0;
+            const int32_t *sc = reinterpret_cast<const int32_t *>(stage + L.rv) + line_off(colind + e0) - e0;
+            for (int t = t0; t < t1; t += kStage) {
+                T v[kStage], xv[kStage];
+#pragma unroll
+                for (int u2 = 0; u2 < kStage; ++u2) {
+                    v[u2] = T(0);
+                    xv[u2] = T(0);
+                    if (t + u2 < t1) {
+                        const int q = SLA_IDX(t + u2 - e0, cap + 4, kBndLocal) + e0;
+                        v[u2] = sv[q];
+                        xv[u2] = __ldg(xb + SLA_IDX(sc[q], x_stride, kBndColumn));
+                    }
+                }
+#pragma unroll
+                for (int u2 = 0; u2 < kStage; ++u2)
+                    if (t + u2 < t1) s += v[u2] * xv[u2];
+            }
+        } else {
+            for (int t = t0; t < t1; ++t) {
+                const int tt = SLA_IDX(t, nnz, kBndEntry);
+                s += __ldg(vb + tt) * __ldg(xb + SLA_IDX(__ldg(colind + tt), x_stride, kBndColumn));
+            }
+        }
+        T *yb = y + (int64_t)sys * n_rows;
+        yb[i] = (beta == T(0)) ? alpha * s : alpha * s + beta * yb[i];
+    }
+    cp_async_wait<0>();
+}
+
 // grad[t] = -(lambda[i] * x[colind[t]]) for entry t of row i, or +(u[i] x[...])
 // when NEG is false (+= if accumulate); LANES threads a row.
 template <typename T, int LANES, bool NEG>
@@ -208,11 +372,11 @@ grad_warp_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__re
         const T *xb = x + (int64_t)sys * n_cols;
         T *gb = grad + (int64_t)sys * nnz;
         if (staged) {
-            for (int base = e0 + lane; base < e1; base += 32 * kStage) {
-                int c[kStage];
-                T li[kStage], xv[kStage], old[kStage];
+            for (int base = e0 + lane; base < e1; base += 32 * kGradStage) {
+                int c[kGradStage];
+                T li[kGradStage], xv[kGradStage], old[kGradStage];
 #pragma unroll
-                for (int u = 0; u < kStage; ++u) {
+                for (int u = 0; u < kGradStage; ++u) {
                     const int t = base + 32 * u;
                     c[u] = 0;
                     li[u] = T(0);
@@ -225,9 +389,9 @@ grad_warp_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__re
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < kStage; ++u) xv[u] = base + 32 * u < e1 ? __ldg(xb + c[u]) : T(0);
+                for (int u = 0; u < kGradStage; ++u) xv[u] = base + 32 * u < e1 ? __ldg(xb + c[u]) : T(0);
 #pragma unroll
-                for (int u = 0; u < kStage; ++u) {
+                for (int u = 0; u < kGradStage; ++u) {
                     const int t = base + 32 * u;
                     if (t < e1) {
                         const T p = mul_rn(li[u], xv[u]);   // rounded on its own, never fused
@@ -251,6 +415,40 @@ grad_warp_kernel(int n_rows, int n_cols, int64_t nnz, int B, const int32_t *__re
 static dim3 row_grid(int rows, int lanes, int B) {
     const int rpb = kRowBlock / lanes;
     return dim3((unsigned)((rows + rpb - 1) / rpb), (unsigned)(B < 65535 ? B : 65535));
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
+// The pipelined SpMV runs for fp64 values (fp32 measured faster with one chunk
+// a block) and needs 16-byte aligned pattern arrays and per-system value
+// arrays; SLA_SPMV_PIPE=0 turns it off.
+static bool pipe_ok(const Csr *h, const void *vals) {
+    const char *e = getenv("SLA_SPMV_PIPE");
+    if ((e && e[0] == '0') || h->dtype != SLA_F64 || !aligned16(h->rowptr) || !aligned16(h->colind))
+        return false;
+    return aligned16(vals) && (h->batch == 1 || (h->nnz * (int64_t)sizeof(double)) % 16 == 0);
+}
+
+// Resident blocks of the pipelined kernel: SMs x blocks an SM holds with
+// `smem` bytes each (computed on first use and kept in the handle).
+template <typename K>
+static sla_status pipe_grid(K kernel, size_t smem, int32_t *cached, int *out) {
+    if (*cached == 0) {
+        SLA_CHECK_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        int per_sm = 0, dev = 0, sms = 0;
+        SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kChunkRows, smem));
+        SLA_CHECK_CUDA(cudaGetDevice(&dev));
+        SLA_CHECK_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+        SLA_REQUIRE(per_sm > 0, "pipelined kernel: %zu bytes of shared memory do not fit an SM", smem);
+        *cached = per_sm * sms;
+    }
+    *out = *cached;
+    return SLA_OK;
+}
+
+static int pipe_blocks(int grid, int rows, int B) {
+    const int64_t units = (int64_t)((rows + kChunkRows - 1) / kChunkRows) * B;
+    return (int)(units < grid ? units : grid);
 }
 
 template <bool NEG>
@@ -318,6 +516,18 @@ extern "C" sla_status sla_spmv(sla_csr_t hh, const void *vals, const void *x, vo
     const int32_t *rp = use_perm ? h->rowptrT : h->rowptr;
     const int32_t *ci = use_perm ? h->colindT : h->colind;
     const int lanes = use_perm ? lanes_for_mean(rows ? (double)h->nnz / rows : 0.0) : h->lanes;
+    if (!use_perm && lanes == 1 && pipe_ok(h, vals)) {
+        const int cap = chunk_cap(h->row_mean);
+        const size_t smem = (size_t)kPipe * PipeStage(cap, (int)sizeof(double)).bytes();
+        int grid = 0;
+        const sla_status st = pipe_grid(spmv_pipe_kernel<double>, smem, &h->pipe_grid_spmv, &grid);
+        if (st != SLA_OK) return st;
+        spmv_pipe_kernel<double><<<pipe_blocks(grid, rows, h->batch), kChunkRows, smem, s>>>(
+            rows, h->nnz, xlen, h->batch, rp, ci, (const double *)vals, (const double *)x, (double *)y, alpha,
+            beta, cap);
+        SLA_CHECK_LAUNCH();
+        return SLA_OK;
+    }
     if (!use_perm && lanes == 1) {
         const dim3 grid = chunk_grid(rows, h->batch);
         const int cap = chunk_cap(h->row_mean);

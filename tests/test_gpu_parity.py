@@ -190,8 +190,11 @@ def _skewed_csr(seed, n_rows, n_cols):
     return rp, cols
 
 
-def test_spmv_and_gradients_on_skewed_short_rows():
-    """Chunks staged in shared memory and chunks too long for it, in one launch."""
+@pytest.mark.parametrize("pipe", ["1", "0"])
+def test_spmv_and_gradients_on_skewed_short_rows(pipe, monkeypatch):
+    """Chunks staged in shared memory and chunks too long for it, in one launch
+    (the pipelined fp64 SpMV, or one chunk a block)."""
+    monkeypatch.setenv("SLA_SPMV_PIPE", pipe)
     n_rows, n_cols, B = 6000, 5000, 2
     rp, ci = _skewed_csr(11, n_rows, n_cols)
     A = make(rp, ci, B=B, symmetric=False, n_cols=n_cols)
@@ -208,8 +211,10 @@ def test_spmv_and_gradients_on_skewed_short_rows():
     assert np.array_equal(H(A.matvec_grad_values(T(lam), T(x))), -O.grad_values(rp, ci, lam, x))
 
 
-@pytest.mark.parametrize("per_row", [5, 30, 60, 120, 250, 500])
-def test_spmv_parity_all_row_widths(per_row):
+@pytest.mark.parametrize("per_row,pipe", [(5, "1"), (5, "0"), (30, "1"), (60, "1"), (120, "1"), (250, "1"),
+                                          (500, "1")])
+def test_spmv_parity_all_row_widths(per_row, pipe, monkeypatch):
+    monkeypatch.setenv("SLA_SPMV_PIPE", pipe)
     n_rows, n_cols = 3001, 2503
     rp, ci = _random_csr(per_row, n_rows, n_cols, per_row // 2 + 1)
     B = 2
@@ -247,6 +252,20 @@ def test_spmv_alpha_beta():
     L.sla_spmv(A.handle, T(v[None, :]), T(x[None, :]), y, 0, 2.0, -0.5)
     ref = 2.0 * O.spmv(rp, ci, v, x) - 0.5 * y0
     assert rel(H(y)[0], ref) < 1e-15
+
+
+def test_spmv_values_off_the_16_byte_grid():
+    """Values whose address is not a multiple of 16 bytes take the one-chunk-a-block kernel."""
+    rp, ci, v = W.poisson2d(40)
+    A = make(rp, ci)
+    x = W.uniform(5, W.STREAM_B, 1600, -1, 1)
+    buf = torch.zeros(ci.shape[0] + 1, dtype=torch.float64, device=DEV)
+    vals = buf[1:]
+    vals.copy_(T(v))
+    assert vals.data_ptr() % 16 == 8
+    y = H(A.spmv(vals[None, :], T(x[None, :])))[0]
+    bound = _spmv_bound(rp, ci, v, x) * 64 * np.finfo(np.float64).eps + 1e-300
+    assert np.all(np.abs(y - O.spmv(rp, ci, v, x)) <= bound)
 
 
 # ------------------------------------------------------------ gradients ----
