@@ -75,6 +75,7 @@ struct CgArgs {
     const SellRec<T> *sell_rec;             // or [B][sell_nnz] value-and-column records
     int64_t sell_nnz;
     int sell_w;         // > 0: every slice of the sliced layout is sell_w entries wide
+    int sell_pipe;      // on-chip SpMV of widths 5 and 7: next row's columns loaded ahead
     const int32_t *sell_perm;   // or null: the row at each position of the sliced layout
     const int16_t *sell_d16;    // or null: the sliced layout's columns as offsets from their row
 };
@@ -292,6 +293,59 @@ __device__ __forceinline__ double sell_tile_hbm(const CgArgs<T> &a, const T *sva
     return acc;
 }
 
+// sell_tile_hbm for slices all W wide with 16-bit columns: the next row's
+// position and column offsets load while the current row gathers.
+template <int W, int NT, typename T>
+__device__ __forceinline__ double sell_tile_hbm_w(const CgArgs<T> &a, const T *svals, const T *pg, T *qg,
+                                                  int r0, int r1) {
+    double acc = 0.0;
+    int i = r0 + threadIdx.x;
+    if (i >= r1) return acc;
+    int rown = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i), a.n, kBndLocal) : i;
+    int dn[W];
+    sell_d16_fetch<W, 1>(a.sell_d16, i, a.sell_nnz, dn);
+    for (; i < r1; i += NT) {
+        const int row = rown;
+        int d[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) d[k] = dn[k];
+        if (i + NT < r1) {
+            rown = a.sell_perm ? SLA_IDX(__ldg(a.sell_perm + i + NT), a.n, kBndLocal) : i + NT;
+            sell_d16_fetch<W, 1>(a.sell_d16, i + NT, a.sell_nnz, dn);
+        }
+        const T qi = sell_row_w<W, 1>(svals, pg, d, i, row, a.n, a.sell_nnz);
+        qg[row] = qi;
+        acc += (double)pg[row] * (double)qi;
+    }
+    return acc;
+}
+
+// Phase A of the on-chip solver for a tile whose sliced rows are all W wide
+// with 16-bit columns: q of the thread's rows into qreg, returning its part
+// of p.q; the next row's column offsets load while the current row gathers.
+template <int W, int RPT, int NT, typename T>
+__device__ __forceinline__ double onchip_rows_w(const CgArgs<T> &a, const T *svals, const T *pg, int r0,
+                                                int r1, T (&qreg)[RPT]) {
+    const int tid = threadIdx.x;
+    double acc = 0.0;
+    int dn[W];
+    if (r0 + tid < r1) sell_d16_fetch<W>(a.sell_d16, r0 + tid, a.sell_nnz, dn);
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+        const int i = r0 + tid + j * NT;
+        int d[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) d[k] = dn[k];
+        if (j + 1 < RPT && i + NT < r1) sell_d16_fetch<W>(a.sell_d16, i + NT, a.sell_nnz, dn);
+        if (i < r1) {
+            const T qi = sell_row_w<W>(svals, pg, d, i, i, a.n, a.sell_nnz);
+            qreg[j] = qi;
+            acc += (double)pg[i] * (double)qi;
+        }
+    }
+    return acc;
+}
+
 // Every block owns the tiles blockIdx.x + lt * gridDim.x (lt = 0, 1, ...) for
 // the whole solve and takes the decisions (breakdown, stop, alpha, beta) for
 // them itself from the shared partials; ONCHIP keeps x, r and M^-1 of its one
@@ -459,6 +513,10 @@ cg_grid_kernel(CgArgs<T> a) {
                             acc[0] += (double)pg[i] * (double)qi;
                         }
                     }
+                } else if (a.sell_d16 && a.sell_w == 5 && a.sell_pipe) {
+                    acc[0] = onchip_rows_w<5, RPT, NT>(a, a.sell_vals + (int64_t)s * a.sell_nnz, pg, r0, r1, qreg);
+                } else if (sizeof(T) == 4 && a.sell_d16 && a.sell_w == 7 && a.sell_pipe) {
+                    acc[0] = onchip_rows_w<7, RPT, NT>(a, a.sell_vals + (int64_t)s * a.sell_nnz, pg, r0, r1, qreg);
                 } else {
                     const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
 #pragma unroll
@@ -497,7 +555,12 @@ cg_grid_kernel(CgArgs<T> a) {
                     }
                 } else {
                     const T *svals = a.sell_vals + (int64_t)s * a.sell_nnz;
-                    acc[0] = sell_tile_hbm<NT>(a, svals, pg, qg, r0, r1);
+                    if (a.sell_d16 && a.sell_w == 7 && a.sell_pipe)
+                        acc[0] = sell_tile_hbm_w<7, NT>(a, svals, pg, qg, r0, r1);
+                    else if (a.sell_d16 && a.sell_w == 5 && a.sell_pipe)
+                        acc[0] = sell_tile_hbm_w<5, NT>(a, svals, pg, qg, r0, r1);
+                    else
+                        acc[0] = sell_tile_hbm<NT>(a, svals, pg, qg, r0, r1);
                 }
             } else {
                 T *qg = a.q + (int64_t)s * n;
@@ -768,6 +831,28 @@ cg_grid2_kernel(CgArgs<T> a) {
         const T *pprev = pbuf[k & 1];
         T *pcur = pbuf[(k + 1) & 1];
         double acc[1] = {0.0};
+        if (a.sell_d16 && a.sell_w == 5 && a.sell_pipe) {
+            // the next row's column offsets load while this row gathers
+            int dn[5];
+            if (r0 + tid < r1) sell_d16_fetch<5>(a.sell_d16, r0 + tid, a.sell_nnz, dn);
+#pragma unroll
+            for (int j = 0; j < RPT; ++j) {
+                const int i = r0 + tid + j * NT;
+                int d[5];
+#pragma unroll
+                for (int k = 0; k < 5; ++k) d[k] = dn[k];
+                if (j + 1 < RPT && i + NT < r1) sell_d16_fetch<5>(a.sell_d16, i + NT, a.sell_nnz, dn);
+                if (i < r1) {
+                    const T qi = sell_row_dir_w<5>(svals, zg, pprev, bt, d, i, a.n, a.sell_nnz);
+                    qreg[j] = qi;
+                    T pi;
+                    if constexpr (sizeof(T) == 8) pi = __fma_rn(bt, pprev[i], __dmul_rn(ds[i - r0], rs[i - r0]));
+                    else pi = __fmaf_rn(bt, pprev[i], __fmul_rn(ds[i - r0], rs[i - r0]));
+                    pcur[i] = pi;
+                    acc[0] += (double)pi * (double)qi;
+                }
+            }
+        } else {
 #pragma unroll
         for (int j = 0; j < RPT; ++j) {
             const int i = r0 + tid + j * NT;
@@ -784,6 +869,7 @@ cg_grid2_kernel(CgArgs<T> a) {
                 pcur[i] = pi;
                 acc[0] += (double)pi * (double)qi;
             }
+        }
         }
         block_sums<NT, 1>(acc, red);
         if (tid == 0 && has_tile) P0[tile] = acc[0];
@@ -2184,6 +2270,8 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             a.sell_cols = h->sell_cols;
             a.sell_nnz = h->sell_nnz;
             a.sell_w = h->sell_w;
+            const char *sp = getenv("SLA_SELL_PIPE");
+            a.sell_pipe = sp && sp[0] == '0' ? 0 : 1;
             a.sell_perm = h->sell_perm;
             a.sell_d16 = h->sell_d16;
             const char *pk = getenv("SLA_SELL_PACK");

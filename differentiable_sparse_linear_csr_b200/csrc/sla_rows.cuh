@@ -147,8 +147,10 @@ __device__ __forceinline__ void sell_slice(const int32_t *__restrict__ sptr, int
 // the row's entries in stored order, then the slice's zero padding (which adds
 // nothing), so the sum equals row_dot<T, 1>.  One row at a time per thread:
 // interleaving a thread's rows spreads its gathers of v and measured slower,
-// and so did loading a row's entries into registers before gathering (the
-// registers spill at the solver's 64-register budget).  uw > 0: every slice is
+// and so did loading a row's values and columns into registers before
+// gathering (the registers spill at the solver's 64-register budget).  For
+// uniform widths of 5 and 7 the solvers use sell_row_w below, which loads only
+// the next row's column offsets ahead.  uw > 0: every slice is
 // uw wide (no slice offsets read).  i is the row's position in the layout and
 // row the row itself (they differ when windows are sorted); with D16 the
 // columns come from d16 as offsets from row, else from cols.
@@ -164,6 +166,52 @@ __device__ __forceinline__ T sell_row(const int32_t *__restrict__ sptr,
         const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
         const int c = D16 ? row + sell_load_d16<STREAM>(d16 + t) : sell_load<STREAM>(cols + t);
         s += sell_load<STREAM>(vals + t) * v[SLA_IDX(c, ncols, kBndColumn)];
+    }
+    return s;
+}
+
+// Rows of a sliced layout whose slices are all W wide, with 16-bit columns,
+// for a thread that walks several rows: sell_d16_fetch loads a row's column
+// offsets ahead of time, so that while one row's values and gathers are in
+// flight the next row's offsets are too, and a row waits for one dependent
+// load (its gathers) instead of two.  sell_row_w sums the row as sell_row does
+// (stored order, the padding adds zeros), so results are bit-identical.
+template <int W, int STREAM = 0>
+__device__ __forceinline__ void sell_d16_fetch(const int16_t *__restrict__ d16, int i, int64_t nslots,
+                                               int (&d)[W]) {
+    const int base = (i / kSellRows) * kSellRows * W + i % kSellRows;
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+        d[k] = sell_load_d16<STREAM>(d16 + SLA_IDX(base + k * kSellRows, nslots, kBndEntry));
+}
+
+template <int W, int STREAM = 0, typename T>
+__device__ __forceinline__ T sell_row_w(const T *__restrict__ vals, const T *v, const int (&d)[W], int i,
+                                        int row, int ncols, int64_t nslots) {
+    const int base = (i / kSellRows) * kSellRows * W + i % kSellRows;
+    T s = T(0);
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        s += sell_load<STREAM>(vals + t) * v[SLA_IDX(row + d[k], ncols, kBndColumn)];
+    }
+    return s;
+}
+
+// sell_row_dir for slices W wide with the row's column offsets already loaded.
+template <int W, typename T>
+__device__ __forceinline__ T sell_row_dir_w(const T *__restrict__ vals, const T *z, const T *pprev, T beta,
+                                            const int (&d)[W], int i, int ncols, int64_t nslots) {
+    const int base = (i / kSellRows) * kSellRows * W + i % kSellRows;
+    T s = T(0);
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        const int c = SLA_IDX(i + d[k], ncols, kBndColumn);
+        T pj;
+        if constexpr (sizeof(T) == 8) pj = __fma_rn(beta, pprev[c], z[c]);
+        else pj = __fmaf_rn(beta, pprev[c], z[c]);
+        s += __ldg(vals + t) * pj;
     }
     return s;
 }
