@@ -415,6 +415,30 @@ def test_results_are_bitwise_reproducible(onchip, monkeypatch):
         assert torch.equal(x1, x2) and torch.equal(i1.iters, i2.iters)
 
 
+@pytest.mark.parametrize("dtype,onchip,grid2", [(torch.float64, "1", "0"), (torch.float32, "1", "1"),
+                                                (torch.float64, "0", "0"), (torch.float32, "1", "0")])
+def test_row_ahead_column_loads_are_bit_identical(dtype, onchip, grid2, monkeypatch):
+    """Loading the next row's column offsets ahead (uniform widths 5 and 7)
+    changes no result bit: three-phase on chip, two barriers, vectors in HBM."""
+    monkeypatch.setenv("SLA_GRID_ONCHIP", onchip)
+    monkeypatch.setenv("SLA_GRID2", grid2)
+    npdt = np.float64 if dtype == torch.float64 else np.float32
+    w3 = W.c3_diffusion3d(N=40)
+    for rp, ci, v in (W.poisson2d(150), (w3.rowptr, w3.colind, w3.values[0])):
+        n = rp.shape[0] - 1
+        A = make(rp, ci, dtype=dtype)
+        assert A.props.sliced == 2 and A.props.sliced_col_bytes == 2
+        b = T(W.uniform(7, W.STREAM_B, n, -1, 1).astype(npdt)[None, :])
+        vals = T(v.astype(npdt)[None, :])
+        out = {}
+        for pipe in ("1", "0"):
+            monkeypatch.setenv("SLA_SELL_PIPE", pipe)
+            x, info = A.cg(vals, b, fixed_iters=40, strategy=L.SLA_STRATEGY_GRID)
+            lam, _ = A.cg(vals, x, adjoint=True, fixed_iters=40, strategy=L.SLA_STRATEGY_GRID)
+            out[pipe] = (x, lam)
+        assert torch.equal(out["1"][0], out["0"][0]) and torch.equal(out["1"][1], out["0"][1])
+
+
 # ----------------------------------------------------- adjoint + gradient ----
 
 @pytest.mark.parametrize("symmetric_flag", [True, False])
