@@ -764,6 +764,9 @@ def main():
         traffic = profile_traffic(f"cg_kernel_{args.workload}_{args.dtype}", (fwd_it + adj_it) / 2)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                # DRAM bytes of the profile at this launch's time: how busy DRAM is
+                "traffic_gbs": None if traffic is None else traffic / (cg_ms / 2 / 1000.0) / 1e9,
+                "traffic_frac": None if traffic is None else traffic / (cg_ms / 2 / 1000.0) / 1e9 / peak,
                 "kernel": f"PCG solve kernel ({variant}), one launch per solve",
                 "algorithmic_bytes_per_launch": (fwd_it + adj_it) * it_bytes / 2,
                 "bytes_per_iteration": it_bytes,
