@@ -1117,6 +1117,49 @@ __device__ __forceinline__ void il_row(const int32_t *__restrict__ sptr, const i
     }
 }
 
+// il_row for slices all W wide with 16-bit columns (offsets d from row i,
+// loaded ahead by the caller): same entries, order and rounding.
+template <int W, typename T, int BW>
+__device__ __forceinline__ void il_row_w(const T *__restrict__ sv, const T *v, const int (&d)[W], int i,
+                                         T (&q)[BW], int ncols, int64_t nslots) {
+    const int base = (i / kSellRows) * kSellRows * W + i % kSellRows;
+#pragma unroll
+    for (int s = 0; s < BW; ++s) q[s] = T(0);
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+        const int t = SLA_IDX(base + k * kSellRows, nslots, kBndEntry);
+        const int c = SLA_IDX(i + d[k], ncols, kBndColumn);
+        T av[BW], pv[BW];
+        VecLoad<T, BW>::ld(sv + (int64_t)t * BW, av);
+        VecLoad<T, BW>::ld(v + (int64_t)c * BW, pv);
+#pragma unroll
+        for (int s = 0; s < BW; ++s) q[s] += av[s] * pv[s];
+    }
+}
+
+// Phase A of the interleaved solver over a tile whose slices are all W wide
+// with 16-bit columns: the next row's offsets load while this row gathers.
+template <int W, int NT, typename T, int BW>
+__device__ __forceinline__ void il_tile_w(const CgArgs<T> &a, const T *sv, const T *p, T *q, int r0, int r1,
+                                          double (&acc)[BW]) {
+    int i = r0 + threadIdx.x;
+    if (i >= r1) return;
+    int dn[W];
+    sell_d16_fetch<W, 1>(a.sell_d16, i, a.sell_nnz, dn);
+    for (; i < r1; i += NT) {
+        int d[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) d[k] = dn[k];
+        if (i + NT < r1) sell_d16_fetch<W, 1>(a.sell_d16, i + NT, a.sell_nnz, dn);
+        T qv[BW], pv[BW];
+        il_row_w<W>(sv, p, d, i, qv, a.n, a.sell_nnz);
+        VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
+        VecLoad<T, BW>::st(q + (int64_t)i * BW, qv);
+#pragma unroll
+        for (int s = 0; s < BW; ++s) acc[s] += (double)pv[s] * (double)qv[s];
+    }
+}
+
 template <typename T, int BW>
 __global__ void __launch_bounds__(kCgThreads, 2)
 cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, int ntiles) {
@@ -1221,13 +1264,19 @@ cg_grid_il_kernel(CgArgs<T> a, T *xi, const T *bi, double *part, int tile_rows, 
             double acc[BW];
 #pragma unroll
             for (int s = 0; s < BW; ++s) acc[s] = 0.0;
-            for (int i = r0 + tid; i < r1; i += NT) {
-                T qv[BW], pv[BW];
-                il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, p, i, qv, a.n, a.sell_nnz);
-                VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
-                VecLoad<T, BW>::st(q + (int64_t)i * BW, qv);
+            if (a.sell_d16 && a.sell_w == 7 && a.sell_pipe) {
+                il_tile_w<7, NT>(a, sv, p, q, r0, r1, acc);
+            } else if (a.sell_d16 && a.sell_w == 5 && a.sell_pipe) {
+                il_tile_w<5, NT>(a, sv, p, q, r0, r1, acc);
+            } else {
+                for (int i = r0 + tid; i < r1; i += NT) {
+                    T qv[BW], pv[BW];
+                    il_row<T, BW>(a.sell_ptr, a.sell_cols, sv, p, i, qv, a.n, a.sell_nnz);
+                    VecLoad<T, BW>::ld(p + (int64_t)i * BW, pv);
+                    VecLoad<T, BW>::st(q + (int64_t)i * BW, qv);
 #pragma unroll
-                for (int s = 0; s < BW; ++s) acc[s] += (double)pv[s] * (double)qv[s];
+                    for (int s = 0; s < BW; ++s) acc[s] += (double)pv[s] * (double)qv[s];
+                }
             }
             block_sums<NT, BW>(acc, red);
             if (tid == 0 && has_tile)
@@ -1980,10 +2029,15 @@ sla_status cg_configure(Csr *h) {
         h->grid_threads = kCgThreads;
         h->grid_smem = 0;
         layout(h, h->grid_blocks, &h->tile_rows, &h->ntiles);
-        // batches of 2 or 4 systems: the interleaved solver (values [entry][system])
+        // fp32 batches of 2 or 4 systems: the interleaved solver (values
+        // [entry][system]).  fp64 batches run batch-major, which measured
+        // faster once rows load their column offsets a row ahead (4 x 128^3:
+        // 14.3 k against 8.7 k system-iterations/s); SLA_INTERLEAVE=1 or 0
+        // forces the choice.
         const char *ie = getenv("SLA_INTERLEAVE");
+        const bool want_il = ie ? ie[0] == '1' : h->dtype == SLA_F32;
         h->il_blocks = 0;
-        if ((h->batch == 2 || h->batch == 4) && n > 0 && !(ie && ie[0] == '0')) {
+        if ((h->batch == 2 || h->batch == 4) && n > 0 && want_il) {
             const void *f = pick_il(h->dtype, h->batch);
             int per_il = 0;
             SLA_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_il, f, kCgThreads, 0));
@@ -2256,6 +2310,10 @@ static sla_status launch_cg(Csr *h, const int32_t *rowptr, const int32_t *colind
             a.sell_cols = h->sell_cols;
             a.sell_vals = sv;
             a.sell_nnz = h->sell_nnz;
+            a.sell_w = h->sell_w;
+            a.sell_d16 = h->sell_d16;
+            const char *sp = getenv("SLA_SELL_PIPE");
+            a.sell_pipe = sp && sp[0] == '0' ? 0 : 1;
             SLA_CHECK_CUDA(cudaMemsetAsync(a.sync, 0, 16 * sizeof(unsigned), s));
             const T *bic = bi;
             void *args[] = {&a, &xi, &bic, &part, (void *)&tile_rows, (void *)&ntiles};

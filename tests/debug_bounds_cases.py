@@ -112,7 +112,10 @@ def main():
              strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0"})
     w = W.c3_batched(N=24, B=2)
     pipeline("interleaved batch of 2", w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,
-             strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0"})
+             strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0", "SLA_INTERLEAVE": "1"})
+    pipeline("interleaved batch of 2, per-slice widths", w.rowptr, w.colind, w.values, w.b, w.xstar,
+             fixed_iters=30, strategy=L.SLA_STRATEGY_GRID,
+             env={"SLA_GRID_ONCHIP": "0", "SLA_INTERLEAVE": "1", "SLA_SELL_UNIFORM": "0"})
     # a non-symmetric pattern: adjoint and SpMV through A^T's pattern
     rp, ci, v = W.random_spd(1500, 0.004, 5, diag_extra=0.5)
     pipeline("adjoint through the transposed pattern", rp, ci, v[None, :], W.normal(5, 0, 1500)[None, :],

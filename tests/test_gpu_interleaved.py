@@ -130,3 +130,33 @@ def test_bounded_wait_times_out_without_hanging(monkeypatch):
     xo, _ = O.pcg(w.rowptr, w.colind, w.values, w.b, fixed_iters=20)
     assert np.all(H(info.status) == L.SLA_FIXED_DONE)
     assert max(rel(H(x)[s], xo[s]) for s in range(2)) < 1e-8
+
+
+@pytest.mark.parametrize("B", [2, 4])
+@pytest.mark.parametrize("dtype", [torch.float64, torch.float32])
+def test_row_ahead_column_loads_are_bit_identical(B, dtype, monkeypatch):
+    """Uniform 7-wide slices with 16-bit columns: loading the next row's column
+    offsets ahead changes no result bit."""
+    npdt = np.float64 if dtype == torch.float64 else np.float32
+    w = W.c3_batched(N=32, B=B)
+    A = _make(w, dtype, monkeypatch)
+    assert A.props.interleaved == 1 and A.props.sliced == 2 and A.props.sliced_col_bytes == 2
+    v, b = T(w.values.astype(npdt)), T(w.b.astype(npdt))
+    out = {}
+    for pipe in ("1", "0"):
+        monkeypatch.setenv("SLA_SELL_PIPE", pipe)
+        out[pipe], _ = A.cg(v, b, fixed_iters=40, strategy=GRID)
+    assert torch.equal(out["1"], out["0"])
+    xo, _ = O.pcg(w.rowptr, w.colind, w.values.astype(npdt), w.b.astype(npdt), fixed_iters=40)
+    tol = 1e-8 if dtype == torch.float64 else 1e-4
+    for s in range(B):
+        assert rel(H(out["1"])[s], xo[s]) < tol
+
+
+def test_fp64_batches_default_to_batch_major(monkeypatch):
+    monkeypatch.setenv("SLA_GRID_ONCHIP", "0")
+    monkeypatch.delenv("SLA_INTERLEAVE", raising=False)
+    w = W.c3_batched(N=13, B=2)
+    A64 = sla.CSR(T(w.rowptr), T(w.colind), batch=2, dtype=torch.float64, symmetric=True)
+    A32 = sla.CSR(T(w.rowptr), T(w.colind), batch=2, dtype=torch.float32, symmetric=True)
+    assert A64.props.interleaved == 0 and A32.props.interleaved == 1
