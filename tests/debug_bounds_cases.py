@@ -8,7 +8,8 @@ block per system with and without the matrix in shared memory, persistent grid
 with vectors on chip or in HBM, tile flags or a third barrier, sliced (uniform or
 per-slice widths, rows sorted within windows, 16- or 32-bit columns) or CSR
 rows, two-barrier form, the
-interleaved batch, lists of systems, the allocation-free entry point), the
+interleaved batch, rows loading their column offsets a row ahead, lists of
+systems, the allocation-free entry point), the
 adjoints (symmetric and through A^T's pattern), SpMV both ways, both value
 gradients and the edge-weighted Laplacian; compares each result with the CPU
 oracle and requires a clean bounds record.  Then plants one out-of-range
@@ -110,12 +111,21 @@ def main():
     pipeline("irregular rows, vectors in HBM, sorted windows", rp, ci, v[None, :],
              W.uniform(8, 0, 12000, -1, 1)[None, :], W.uniform(8, 1, 12000, -1, 1)[None, :], fixed_iters=30,
              strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0"})
-    w = W.c3_batched(N=24, B=2)
+    w = W.c3_batched(N=32, B=2)   # uniform 7-wide slices: columns loaded a row ahead
     pipeline("interleaved batch of 2", w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,
              strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0", "SLA_INTERLEAVE": "1"})
     pipeline("interleaved batch of 2, per-slice widths", w.rowptr, w.colind, w.values, w.b, w.xstar,
              fixed_iters=30, strategy=L.SLA_STRATEGY_GRID,
              env={"SLA_GRID_ONCHIP": "0", "SLA_INTERLEAVE": "1", "SLA_SELL_UNIFORM": "0"})
+    pipeline("batch of 2 in HBM, batch-major", w.rowptr, w.colind, w.values, w.b, w.xstar, fixed_iters=30,
+             strategy=L.SLA_STRATEGY_GRID, env={"SLA_GRID_ONCHIP": "0", "SLA_INTERLEAVE": "0"})
+    # one 2-D grid on chip with uniform 5-wide slices (columns loaded a row ahead), three
+    # phases with tile flags and the two-barrier form
+    rp, ci, v = W.poisson2d(100)
+    b2, x2 = W.uniform(12, 0, 10000, -1, 1)[None, :], W.uniform(12, 1, 10000, -1, 1)[None, :]
+    for label, env in (("2-D grid on chip, three phases", {"SLA_GRID2": "0"}),
+                       ("2-D grid on chip, two barriers", {"SLA_GRID2": "2"})):
+        pipeline(label, rp, ci, v[None, :], b2, x2, fixed_iters=30, strategy=L.SLA_STRATEGY_GRID, env=env)
     # a non-symmetric pattern: adjoint and SpMV through A^T's pattern
     rp, ci, v = W.random_spd(1500, 0.004, 5, diag_extra=0.5)
     pipeline("adjoint through the transposed pattern", rp, ci, v[None, :], W.normal(5, 0, 1500)[None, :],
