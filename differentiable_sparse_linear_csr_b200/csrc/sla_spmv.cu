@@ -195,11 +195,13 @@ __device__ __forceinline__ void stage_range(uint32_t dst, const void *lo, const 
                                             int tid) {
     const uintptr_t a0 = (uintptr_t)lo & ~(uintptr_t)15;
     const int pieces = (int)(((uintptr_t)hi - a0 + 15) >> 4);
-    for (int q = tid; q < pieces; q += kChunkRows) {
-        const uintptr_t src = a0 + 16 * (uintptr_t)q;
-        const uintptr_t left = (uintptr_t)end - src;
-        cp_async16(dst + 16 * q, (const void *)src, left >= 16 ? 16 : (int)left);
-    }
+    // pieces before `end` that are whole, and the bytes of the one it cuts
+    const uintptr_t room = (uintptr_t)end - a0;
+    const int whole = room >= (uintptr_t)pieces * 16 ? pieces : (int)(room >> 4);
+    const int cut = (int)(room & 15);
+    const char *src = reinterpret_cast<const char *>(a0);
+    for (int q = tid; q < pieces; q += kChunkRows)
+        cp_async16(dst + 16 * q, src + 16 * q, q < whole ? 16 : cut);
 }
 
 // Element offset of p within its 16-byte line.
@@ -245,20 +247,31 @@ spmv_pipe_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32_t
     const PipeStage L(cap, (int)sizeof(T));
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem_raw);
     const int nchunks = (n_rows + kChunkRows - 1) / kChunkRows;
-    const int64_t units = (int64_t)nchunks * B;
-    const int64_t G = gridDim.x;
-    const int mine = blockIdx.x < units ? (int)((units - blockIdx.x + G - 1) / G) : 0;
+    const int units = nchunks * B;     // below 2^31 (checked by the caller)
+    const int G = gridDim.x;
+    const int mine = (int)blockIdx.x < units ? (units - (int)blockIdx.x + G - 1) / G : 0;
+    // system and first row of unit u (no division for one system)
+    auto unit = [&](int u, int &sys, int &r0) {
+        if (B == 1) {
+            sys = 0;
+            r0 = u * kChunkRows;
+        } else {
+            sys = (int)((unsigned)u / (unsigned)nchunks);
+            r0 = (u - sys * nchunks) * kChunkRows;
+        }
+    };
     // entry range of my k-th chunk (read one iteration before its copy is queued)
     auto range = [&](int k, int &e0, int &e1) {
         if (k >= mine) return;
-        const int r0 = (int)((blockIdx.x + k * G) % nchunks) * kChunkRows;
+        int sys, r0;
+        unit((int)blockIdx.x + k * G, sys, r0);
         e0 = SLA_IDX(__ldg(rowptr + r0), nnz + 1, kBndEntry);
         e1 = SLA_IDX(__ldg(rowptr + min(n_rows, r0 + kChunkRows)), nnz + 1, kBndEntry);
     };
     auto issue = [&](int k, int e0, int e1) {
         if (k >= mine) return;
-        const int64_t u = blockIdx.x + k * G;
-        const int sys = (int)(u / nchunks), r0 = (int)(u % nchunks) * kChunkRows;
+        int sys, r0;
+        unit((int)blockIdx.x + k * G, sys, r0);
         pipe_issue<T>(sbase + (k % kPipe) * L.bytes(), L, cap, n_rows, nnz, r0, e0, e1, rowptr, colind,
                       vals + (int64_t)sys * nnz, tid);
     };
@@ -276,8 +289,8 @@ spmv_pipe_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32_t
         issue(j + kPipe - 1, ne0, ne1);
         cp_async_commit();
         range(j + kPipe, ne0, ne1);
-        const int64_t u = blockIdx.x + j * G;
-        const int sys = (int)(u / nchunks), r0 = (int)(u % nchunks) * kChunkRows;
+        int sys, r0;
+        unit((int)blockIdx.x + j * G, sys, r0);
         const int r1 = min(n_rows, r0 + kChunkRows), i = r0 + tid;
         unsigned char *stage = smem_raw + (j % kPipe) * L.bytes();
         const int32_t *srp = reinterpret_cast<const int32_t *>(stage + L.rv + L.rc) + line_off(rowptr + r0);
@@ -426,6 +439,7 @@ static bool pipe_ok(const Csr *h, const void *vals) {
     const char *e = getenv("SLA_SPMV_PIPE");
     if ((e && e[0] == '0') || h->dtype != SLA_F64 || !aligned16(h->rowptr) || !aligned16(h->colind))
         return false;
+    if ((int64_t)((h->n_rows + kChunkRows - 1) / kChunkRows) * h->batch >= INT32_MAX) return false;
     return aligned16(vals) && (h->batch == 1 || (h->nnz * (int64_t)sizeof(double)) % 16 == 0);
 }
 
