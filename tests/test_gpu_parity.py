@@ -254,6 +254,26 @@ def test_spmv_alpha_beta():
     assert rel(H(y)[0], ref) < 1e-15
 
 
+@pytest.mark.parametrize("B", [1, 3])
+def test_pipelined_spmv_batches_and_alpha_beta(B):
+    """The pipelined fp64 SpMV over several systems (each system's values on the
+    16-byte grid: 7840 entries), with y = alpha A x + beta y."""
+    rp, ci, v = W.poisson2d(40)
+    n, nnz = 1600, ci.shape[0]
+    assert (nnz * 8) % 16 == 0
+    A = make(rp, ci, B=B)
+    vals = W.uniform(13, W.STREAM_WEIGHTS, B * nnz, -1, 1).reshape(B, nnz)
+    x = W.uniform(13, W.STREAM_B, B * n, -1, 1).reshape(B, n)
+    y0 = W.uniform(14, W.STREAM_B, B * n, -1, 1).reshape(B, n)
+    y = T(y0).clone()
+    L.sla_spmv(A.handle, T(vals), T(x), y, 0, 1.5, -0.25)
+    for s_ in range(B):
+        ref = 1.5 * O.spmv(rp, ci, vals[s_], x[s_]) - 0.25 * y0[s_]
+        eps = np.finfo(np.float64).eps
+        bound = (1.5 * _spmv_bound(rp, ci, vals[s_], x[s_]) * 64 + 0.25 * np.abs(y0[s_]) * 4) * eps + 1e-300
+        assert np.all(np.abs(H(y)[s_] - ref) <= bound)
+
+
 def test_spmv_values_off_the_16_byte_grid():
     """Values whose address is not a multiple of 16 bytes take the one-chunk-a-block kernel."""
     rp, ci, v = W.poisson2d(40)
