@@ -39,6 +39,9 @@
  *   - Workspace is caller-provided device memory of at least
  *     sla_workspace_bytes() bytes, 256-byte aligned.  Solves and SpMVs never
  *     allocate device memory.  Concurrent calls need distinct workspaces.
+ *   - A handle fills a few caches on first use (A^T's pattern for a
+ *     non-symmetric handle, the resident grid of the pipelined SpMV); calls on
+ *     one handle from several host threads must be serialised by the caller.
  *   - Every device-side wait is bounded (sla_cg_opts.wait_timeout_ns); a wait
  *     that runs out makes the kernel return and the affected systems report
  *     SLA_TIMED_OUT.  No kernel traps.
