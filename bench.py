@@ -63,13 +63,29 @@ def edge_metrics(n: int, nnz: int, E: int, B: int, vbytes: int, asm_ms: float, g
             "edge_grad_gbs": grad_bytes_ / (grad_ms / 1000.0) / 1e9}
 
 
-def source_digest() -> str:
+def source_digest(files=None) -> str:
+    """sha256 (16 hex digits) of the library source: every file of csrc/, or
+    only `files` (names in csrc/), those a profiled kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_sparse_linear_csr_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files else os.listdir(csrc)):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
+
+
+def profile_digest_matches(text: str) -> bool:
+    """A summary's `source_digest` against the current source: over the files
+    its `source_files` line names when it has one (the profiled kernel's own
+    sources), else over all of csrc/."""
+    d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    if not d:
+        return False
+    f = re.search(r"^source_files:\s*(.+)$", text, re.M)
+    try:
+        return d.group(1) == source_digest(f.group(1).split() if f else None)
+    except OSError:
+        return False
 
 
 def profile_traffic(kernel_key: str, iters_per_launch: float):
@@ -81,8 +97,7 @@ def profile_traffic(kernel_key: str, iters_per_launch: float):
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
-    if not d or d.group(1) != source_digest():
+    if not profile_digest_matches(text):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if m:

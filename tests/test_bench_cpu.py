@@ -2,7 +2,8 @@
 model against the per-iteration figures of the two-pass model for the
 1024x1024 Poisson (fp64 and fp32) and 128^3 diffusion systems, the rule that
 a committed ncu traffic figure is used only while the library source matches
-it, and clock sampling that degrades to "no samples" without a GPU."""
+it (all of it, or the files the profiled kernel is built from), and clock
+sampling that degrades to "no samples" without a GPU."""
 import os
 
 import pytest
@@ -27,7 +28,7 @@ def _profile(tmp_path, key, body):
 
 def test_traffic_is_used_only_for_the_matching_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "source_digest", lambda: "abc123")
+    monkeypatch.setattr(bench, "source_digest", lambda files=None: "abc123")
     _profile(tmp_path, "k_launch", "traffic_bytes_per_launch: 1.5e9\nsource_digest: abc123\n")
     _profile(tmp_path, "k_iter", "traffic_bytes_per_iteration: 200\nsource_digest: abc123\n")
     _profile(tmp_path, "k_stale", "traffic_bytes_per_iteration: 200\nsource_digest: ffff00\n")
@@ -37,6 +38,33 @@ def test_traffic_is_used_only_for_the_matching_source(tmp_path, monkeypatch):
     assert bench.profile_traffic("k_stale", 924) is None
     assert bench.profile_traffic("k_none", 924) is None
     assert bench.profile_traffic("k_missing", 924) is None
+
+
+def test_traffic_digest_scoped_to_the_kernel_files(tmp_path, monkeypatch):
+    """A summary that names its kernel's source files stays valid while other
+    library files change, and goes stale when one of its own files does."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    csrc = tmp_path / "differentiable_sparse_linear_csr_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "solver.cu").write_text("solver v1")
+    (csrc / "common.cuh").write_text("common v1")
+    (csrc / "other.cu").write_text("other v1")
+    d = bench.source_digest(["solver.cu", "common.cuh"])
+    _profile(tmp_path, "k", f"traffic_bytes_per_iteration: 100\nsource_digest: {d}\n"
+                            "source_files: solver.cu common.cuh\n")
+    assert bench.profile_traffic("k", 10) == 1000
+    (csrc / "other.cu").write_text("other v2")
+    assert bench.profile_traffic("k", 10) == 1000
+    (csrc / "common.cuh").write_text("common v2")
+    assert bench.profile_traffic("k", 10) is None
+    # a summary without a file list is checked against every file
+    _profile(tmp_path, "k_all", f"traffic_bytes_per_iteration: 100\nsource_digest: {bench.source_digest()}\n")
+    assert bench.profile_traffic("k_all", 10) == 1000
+    (csrc / "other.cu").write_text("other v3")
+    assert bench.profile_traffic("k_all", 10) is None
+    # a named file that does not exist makes the figure unusable, not an error
+    _profile(tmp_path, "k_gone", f"traffic_bytes_per_iteration: 100\nsource_digest: {d}\nsource_files: gone.cu\n")
+    assert bench.profile_traffic("k_gone", 10) is None
 
 
 def test_source_digest_covers_the_library_source():
