@@ -390,8 +390,7 @@ def spmv_block(A, vals, n: int, nnz: int, B: int, vbytes: int, dt, dev, flush, p
     read_gbs = by / (ms_read / 1000.0) / 1e9
     del buf
     kernel = ("sla_spmv, pipelined one-thread rows: 256-row chunks copied to shared memory one chunk "
-              "ahead (cp.async)" if vbytes == 8 else
-              "sla_spmv, one-thread rows: 256-row chunks staged in shared memory")
+              "ahead (cp.async)" if A.props.lanes == 1 else "sla_spmv, sub-warp rows")
     return {"ms": ms, "algorithmic_bytes": by, "gbs": gbs, "frac_of_hbm_peak": gbs / peak,
             "same_bytes_read_gbs": read_gbs, "frac_of_same_bytes_read": gbs / read_gbs,
             "same_bytes_read": "torch.sum over a buffer of the same bytes, same flush before each",

@@ -12,7 +12,8 @@
 //    the row in global memory).  Gathering row by row keeps a warp's gathers of
 //    x together for banded patterns (consecutive rows reach consecutive
 //    columns); gathering entry by entry measured slower.
-//    fp64 values take a pipelined form of this (after the staged kernel).
+//    Resident blocks run a pipelined form of this when the arrays are on the
+//    16-byte grid (after the staged kernel).
 //  - Value gradients: each warp takes 32 rows and walks their entry range in
 //    order, the row of each entry taken from a per-warp table, so column reads
 //    and gradient stores are coalesced.
@@ -157,7 +158,7 @@ spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32
     }
 }
 
-// ---- pipelined one-thread-row SpMV (fp64) --------------------------------
+// ---- pipelined one-thread-row SpMV ----------------------------------------
 // A block stays resident and takes the chunks (kChunkRows consecutive rows of
 // one system) blockIdx.x, blockIdx.x + gridDim.x, ... .  A chunk's entries are
 // one contiguous range of the CSR arrays: its values, columns and row pointers
@@ -168,9 +169,9 @@ spmv_staged_kernel(int n_rows, int64_t nnz, int64_t x_stride, int B, const int32
 // down to 16 (the arrays start on 16-byte boundaries) and reads nothing past
 // the array's end.  A chunk with more entries than a stage holds walks its
 // rows in global memory (its row pointers are still staged).  Two stages keep
-// three blocks (24 warps) on an SM for rows of 7; three stages (two chunks
-// ahead) left room for two blocks and measured slower, and so did the same
-// pipeline for the value gradient and for fp32 SpMV on the 2-D Poisson matrix.
+// three blocks (24 warps) on an SM for rows of 7 in fp64; three stages (two
+// chunks ahead) left room for two blocks and measured slower, and so did the
+// same pipeline for the value gradient.
 
 constexpr int kPipe = 2;                 // stages: the chunk in flight + the one being summed
 
@@ -432,15 +433,13 @@ static dim3 row_grid(int rows, int lanes, int B) {
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
-// The pipelined SpMV runs for fp64 values (fp32 measured faster with one chunk
-// a block) and needs 16-byte aligned pattern arrays and per-system value
+// The pipelined SpMV needs 16-byte aligned pattern arrays and per-system value
 // arrays; SLA_SPMV_PIPE=0 turns it off.
 static bool pipe_ok(const Csr *h, const void *vals) {
     const char *e = getenv("SLA_SPMV_PIPE");
-    if ((e && e[0] == '0') || h->dtype != SLA_F64 || !aligned16(h->rowptr) || !aligned16(h->colind))
-        return false;
+    if ((e && e[0] == '0') || !aligned16(h->rowptr) || !aligned16(h->colind)) return false;
     if ((int64_t)((h->n_rows + kChunkRows - 1) / kChunkRows) * h->batch >= INT32_MAX) return false;
-    return aligned16(vals) && (h->batch == 1 || (h->nnz * (int64_t)sizeof(double)) % 16 == 0);
+    return aligned16(vals) && (h->batch == 1 || (h->nnz * (int64_t)dtype_size(h->dtype)) % 16 == 0);
 }
 
 // Resident blocks of the pipelined kernel: SMs x blocks an SM holds with
@@ -532,13 +531,20 @@ extern "C" sla_status sla_spmv(sla_csr_t hh, const void *vals, const void *x, vo
     const int lanes = use_perm ? lanes_for_mean(rows ? (double)h->nnz / rows : 0.0) : h->lanes;
     if (!use_perm && lanes == 1 && pipe_ok(h, vals)) {
         const int cap = chunk_cap(h->row_mean);
-        const size_t smem = (size_t)kPipe * PipeStage(cap, (int)sizeof(double)).bytes();
+        const size_t smem = (size_t)kPipe * PipeStage(cap, (int)dtype_size(h->dtype)).bytes();
         int grid = 0;
-        const sla_status st = pipe_grid(spmv_pipe_kernel<double>, smem, &h->pipe_grid_spmv, &grid);
+        const sla_status st = h->dtype == SLA_F64
+                                  ? pipe_grid(spmv_pipe_kernel<double>, smem, &h->pipe_grid_spmv, &grid)
+                                  : pipe_grid(spmv_pipe_kernel<float>, smem, &h->pipe_grid_spmv, &grid);
         if (st != SLA_OK) return st;
-        spmv_pipe_kernel<double><<<pipe_blocks(grid, rows, h->batch), kChunkRows, smem, s>>>(
-            rows, h->nnz, xlen, h->batch, rp, ci, (const double *)vals, (const double *)x, (double *)y, alpha,
-            beta, cap);
+        if (h->dtype == SLA_F64)
+            spmv_pipe_kernel<double><<<pipe_blocks(grid, rows, h->batch), kChunkRows, smem, s>>>(
+                rows, h->nnz, xlen, h->batch, rp, ci, (const double *)vals, (const double *)x, (double *)y,
+                alpha, beta, cap);
+        else
+            spmv_pipe_kernel<float><<<pipe_blocks(grid, rows, h->batch), kChunkRows, smem, s>>>(
+                rows, h->nnz, xlen, h->batch, rp, ci, (const float *)vals, (const float *)x, (float *)y,
+                (float)alpha, (float)beta, cap);
         SLA_CHECK_LAUNCH();
         return SLA_OK;
     }
